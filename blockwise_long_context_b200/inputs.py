@@ -1,0 +1,124 @@
+"""Seeded synthetic inputs shaped like the pages' workloads.
+
+This module holds no attention arithmetic: it only draws random tensors.
+Both the CUDA path's tests/benchmark and the fp64 oracle take their inputs
+from here, so they see bit-identical values (the oracle widens them to fp64).
+
+Recipe: ``torch.Generator('cpu').manual_seed(seed)``, ``randn`` in fp32,
+multiplied by the tensor's standard deviation, then rounded to the compute
+dtype (round-to-nearest-even for bf16).  Seeds are
+``1000 + 10 * config_index + tensor_id`` with tensor ids
+q=0, k=1, v=2, do=3, y=4, w_k=5, w_v=6.
+
+The shapes stand in for the LV-XAttn review page's workloads (Llama 3-V,
+long-video cross-attention with S_Q << S_KV, Figure 1 / "The reading"; the
+pages' Video-MME inputs are not available, synthetic Gaussians replace them)
+and for Ring-Attention-style causal self-attention.
+"""
+
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field, replace
+from typing import Optional
+
+import torch
+
+TENSOR_IDS = {"q": 0, "k": 1, "v": 2, "do": 3, "y": 4, "w_k": 5, "w_v": 6}
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    index: int
+    B: int
+    H: int
+    H_kv: int
+    d: int
+    S_Q: int
+    S_KV: int
+    n_blocks: int
+    causal: bool
+    dtype: str                     # "f32" or "bf16"
+    qkv_std: float
+    backward: bool
+    d_embed: int = 0               # > 0: K, V recomputed from y
+    desc: str = field(default="", compare=False)
+
+    @property
+    def torch_dtype(self) -> torch.dtype:
+        return torch.float32 if self.dtype == "f32" else torch.bfloat16
+
+    def scaled(self, **kw) -> "Workload":
+        """Same recipe (seeds, distributions) at other sizes."""
+        return replace(self, **kw)
+
+    def fwd_flops(self) -> float:
+        """4 B H S_Q S_KV d, counting only unmasked (query, key) pairs."""
+        if self.causal:
+            pairs = self.S_Q * (self.S_Q + 1) / 2
+        else:
+            pairs = self.S_Q * self.S_KV
+        return 4.0 * self.B * self.H * pairs * self.d
+
+    def bwd_flops(self) -> float:
+        """Five GEMMs against the forward's two: 2.5x the forward count."""
+        return 2.5 * self.fwd_flops() if self.backward else 0.0
+
+    def kv_flops(self) -> float:
+        return 2.0 * 2.0 * self.B * self.S_KV * self.d_embed * self.H_kv * self.d if self.d_embed else 0.0
+
+
+_R2 = 1.0 / math.sqrt(2.0)
+
+WORKLOADS = {
+    "C0": Workload("C0", 0, B=1, H=1, H_kv=1, d=64, S_Q=128, S_KV=1024, n_blocks=4,
+                   causal=False, dtype="f32", qkv_std=1.0, backward=False,
+                   desc="single-head non-causal cross-attention, fp32, n=4, forward"),
+    "C1": Workload("C1", 1, B=1, H=32, H_kv=8, d=128, S_Q=2048, S_KV=65536, n_blocks=8,
+                   causal=False, dtype="bf16", qkv_std=_R2, backward=False,
+                   desc="Llama-3-V-like GQA cross-attention forward, bf16"),
+    "C2": Workload("C2", 2, B=1, H=32, H_kv=8, d=128, S_Q=2048, S_KV=65536, n_blocks=8,
+                   causal=False, dtype="bf16", qkv_std=_R2, backward=True, d_embed=4096,
+                   desc="C1 forward + backward, K/V recomputed from shared visual features"),
+    "C3": Workload("C3", 3, B=1, H=32, H_kv=32, d=128, S_Q=131072, S_KV=131072, n_blocks=8,
+                   causal=True, dtype="bf16", qkv_std=_R2, backward=True,
+                   desc="causal self-attention forward + backward, n=8 block skipping"),
+    "C4": Workload("C4", 4, B=2, H=16, H_kv=16, d=128, S_Q=512, S_KV=262144, n_blocks=16,
+                   causal=False, dtype="bf16", qkv_std=_R2, backward=True,
+                   desc="long-video cross-attention forward + backward, n=16"),
+}
+
+
+def seed_for(w: Workload, tensor: str) -> int:
+    return 1000 + 10 * w.index + TENSOR_IDS[tensor]
+
+
+def _randn(shape, seed: int, std: float, dtype: torch.dtype) -> torch.Tensor:
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    t = torch.randn(*shape, generator=g, dtype=torch.float32)
+    if std != 1.0:
+        t.mul_(std)
+    return t.to(dtype)
+
+
+def make(w: Workload, tensors=("q", "k", "v"), dtype: Optional[torch.dtype] = None) -> dict:
+    """Host tensors for workload ``w`` (contiguous, CPU)."""
+    dt = dtype or w.torch_dtype
+    out = {}
+    for name in tensors:
+        seed = seed_for(w, name)
+        if name == "q":
+            out[name] = _randn((w.B, w.S_Q, w.H, w.d), seed, w.qkv_std, dt)
+        elif name in ("k", "v"):
+            out[name] = _randn((w.B, w.S_KV, w.H_kv, w.d), seed, w.qkv_std, dt)
+        elif name == "do":
+            out[name] = _randn((w.B, w.S_Q, w.H, w.d), seed, 1.0, dt)
+        elif name == "y":
+            out[name] = _randn((w.B, w.S_KV, w.d_embed), seed, 1.0, dt)
+        elif name in ("w_k", "w_v"):
+            out[name] = _randn((w.d_embed, w.H_kv * w.d), seed, 1.0 / math.sqrt(w.d_embed), dt)
+        else:
+            raise KeyError(name)
+    return out
