@@ -1,0 +1,365 @@
+#!/usr/bin/env python
+"""Benchmark of the blockwise attention hot path on B200.
+
+One step = one pass of the whole path over one synthetic batch of the
+Llama-3-V-like GQA cross-attention workload (B=1, H=32, H_kv=8, d=128,
+S_Q=2048, S_KV=65536, n=8 KV blocks, bf16):
+  K, V = y W_k, y W_v        (K/V recomputation from the shared visual features)
+  partials (O_i, L_i) over the 8 KV blocks, then their merge   (forward)
+  D = rowsum(dO o O), dQ, dK, dV from the stored LSE            (backward)
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lvx|reference]
+
+Prints one JSON line (rank 0).  ``value`` is whole-job TFLOP/s over all
+ranks: counted FLOPs (attention forward 4*B*H*S_Q*S_KV*d, backward 2.5x that,
+K/V recomputation 2*2*B*S_KV*d_embed*H_kv*d) divided by the max-over-ranks
+device time of K steps.  With N > 1 every rank runs its own batch of the same
+shape (weak scaling, no data-path collective).  ``--impl reference`` times
+the fp64 CPU oracle on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd+bwd TFLOP/s and % of B200 dense BF16 peak, 1 GPU"
+WORKLOAD = "C2"
+
+# ncu DRAM traffic of the dominant kernel per launch, with the hash of the
+# source file it was taken from (reported only while the source is unchanged).
+TRAFFIC = {}
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sust=d["bf16_tflops_sustained"],
+                    src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sust=1400.0, src="fallback")
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ["clocks.sm", "clocks.max.sm", "clocks_event_reasons.hw_slowdown",
+              "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
+              "clocks_event_reasons.sw_power_cap"]
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            try:
+                sm.append(float(parts[0])); smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(self.NAMES, parts[2:]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------- CPU oracle baseline
+
+def oracle_sample(w, seconds_hint: float = 20.0):
+    """Times the fp64 oracle on a bounded sample of the workload's step.
+
+    Sample: the same heads, head width and S_KV, with S_Q cut to ``rows``
+    query rows (forward + full textbook backward), plus K/V recomputation of
+    ``rows`` rows of y.  Returns (TFLOP/s of counted work, seconds, description).
+    """
+    import numpy as np
+    import oracle
+    from blockwise_long_context_b200 import inputs
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count() or 1
+    rows = 32
+    sw = w.scaled(S_Q=rows)
+    host = inputs.make(sw, tensors=("q", "k", "v", "do"))
+    q, k, v, do = (host[t].double().numpy() for t in ("q", "k", "v", "do"))
+    kvw = inputs.make(w, tensors=("w_k", "w_v")) if w.d_embed else None
+    t0 = time.perf_counter()
+    oracle.attention_fwd(q, k, v, causal=sw.causal)
+    oracle.attention_bwd(q, k, v, do, causal=sw.causal)
+    flops = sw.fwd_flops() + 2.5 * sw.fwd_flops()
+    if kvw is not None:
+        y = np.random.default_rng(0).standard_normal((rows, w.d_embed))
+        oracle.kv_recompute(y, kvw["w_k"].double().numpy(), kvw["w_v"].double().numpy())
+        flops += 2 * 2 * rows * w.d_embed * w.H_kv * w.d
+    dt = time.perf_counter() - t0
+    desc = (f"fp64 oracle, forward + backward for {rows} of {w.S_Q} query rows over all {w.H} heads "
+            f"and all {w.S_KV} keys, plus K/V recompute of {rows} rows of y; counted FLOPs / time")
+    return flops / dt / 1e12, dt, cores, desc
+
+
+def run_reference(a):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from blockwise_long_context_b200 import inputs
+    w = inputs.WORKLOADS[a.workload]
+    for _ in range(a.warmup):
+        oracle_sample(w)
+    vals, secs = [], []
+    cores, desc = 1, ""
+    for _ in range(a.steps):
+        v, s, cores, desc = oracle_sample(w)
+        vals.append(v); secs.append(s)
+    value = statistics.mean(vals)
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": a.gpus,
+            "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * statistics.mean(secs),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": _config(w, a.gpus),
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def _config(w, n):
+    return {"workload": f"{w.name}: {w.desc}", "B": w.B, "H": w.H, "H_kv": w.H_kv, "d": w.d,
+            "S_Q": w.S_Q, "S_KV": w.S_KV, "n_blocks": w.n_blocks, "causal": w.causal,
+            "d_embed": w.d_embed, "parallelism": f"replicas{n}" if n > 1 else "single",
+            "l2": "inputs larger than L2: y 512 MiB read and K/V 256 MiB rewritten every step",
+            "flops_counted": "attn fwd 4*B*H*S_Q*S_KV*d + bwd 2.5x fwd + K/V recompute "
+                             "2*2*B*S_KV*d_embed*H_kv*d"}
+
+
+# ---------------------------------------------------------------- GPU arm
+
+def _file_sha(rel):
+    p = os.path.join(ROOT, rel)
+    return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16] if os.path.exists(p) else None
+
+
+def run_gpu(a):
+    import torch
+    import torch.distributed as dist
+    from blockwise_long_context_b200 import inputs
+    from blockwise_long_context_b200 import binding as lvx
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    w = inputs.WORKLOADS[a.workload]
+    peaks = _peaks()
+
+    host = inputs.make(w, tensors=("q", "do", "y", "w_k", "w_v"))
+    pinned = {k: t.pin_memory() for k, t in host.items()}
+    d = {k: t.to(dev) for k, t in pinned.items()}
+    B, S_Q, H, hd = d["q"].shape
+    k = torch.empty(w.B, w.S_KV, w.H_kv, w.d, dtype=torch.bfloat16, device=dev)
+    v = torch.empty_like(k)
+    out = torch.empty_like(d["q"])
+    lse = torch.empty(B, H, S_Q, dtype=torch.float32, device=dev)
+    dq = torch.empty_like(d["q"]); dk = torch.empty_like(k); dv = torch.empty_like(k)
+    fws = lvx.fwd_workspace(d["q"], k, w.n_blocks, w.causal)
+    bws = lvx.bwd_workspace(d["q"], k, w.causal)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev: ev[0].record(stream)
+        lvx.lvx_kv_recompute(d["y"], d["w_k"], d["w_v"], k, v, w.H_kv, w.d)
+        if ev: ev[1].record(stream)
+        lvx.lvx_attn_fwd(d["q"], k, v, out, lse, w.n_blocks, w.causal, 0.0, fws)
+        if ev: ev[2].record(stream)
+        lvx.lvx_attn_bwd(d["q"], k, v, out, lse, d["do"], dq, dk, dv, w.causal, 0.0, bws)
+        if ev: ev[3].record(stream)
+
+    warm = max(a.warmup, 3)
+    for _ in range(warm):
+        step()
+    torch.cuda.synchronize()
+    lvx.lvx_last_device_error()
+
+    stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(a.steps)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    e0.record(stream)
+    for i in range(a.steps):
+        step(stage_ev[i])
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    ms_total = e0.elapsed_time(e1)
+    t_kv = statistics.mean(ev[0].elapsed_time(ev[1]) for ev in stage_ev)
+    t_fwd = statistics.mean(ev[1].elapsed_time(ev[2]) for ev in stage_ev)
+    t_bwd = statistics.mean(ev[2].elapsed_time(ev[3]) for ev in stage_ev)
+    lvx.lvx_last_device_error()
+
+    if world > 1:
+        t = torch.tensor([ms_total], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / a.steps
+    step_flops = w.fwd_flops() + w.bwd_flops() + w.kv_flops()
+    value = world * step_flops * a.steps / (ms_total * 1e-3) / 1e12
+
+    # merge kernel alone (HBM-bound), after an L2 flush, through the merge entry point
+    flush = torch.empty(256 * 2**20, dtype=torch.uint8, device=dev)
+    O_p, L_p = lvx.fwd_partials_view(fws, w.n_blocks, w.B, w.H, w.S_Q, w.d)
+    mt = []
+    for _ in range(5):
+        flush.zero_()
+        m0, m1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        m0.record(stream)
+        lvx.lvx_merge_partials(O_p, L_p, out, lse)
+        m1.record(stream)
+        torch.cuda.synchronize()
+        mt.append(m0.elapsed_time(m1))
+    t_merge = statistics.median(mt)
+    merge_bytes = w.B * w.H * w.S_Q * (w.n_blocks * (4 * w.d + 4) + (2 * w.d + 4))
+    merge_gbs = merge_bytes / (t_merge * 1e-3) / 1e9
+
+    # end to end through the public API with host buffers
+    res_host = {"dq": torch.empty(dq.shape, dtype=dq.dtype).pin_memory(),
+                "dk": torch.empty(dk.shape, dtype=dk.dtype).pin_memory(),
+                "dv": torch.empty(dv.shape, dtype=dv.dtype).pin_memory()}
+    h2d = sum(t.numel() * t.element_size() for t in pinned.values())
+    d2h = sum(t.numel() * t.element_size() for t in res_host.values())
+    n_e2e = max(3, min(a.steps, 10))
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    x0.record(stream)
+    for _ in range(n_e2e):
+        for name, t in pinned.items():
+            d[name].copy_(t, non_blocking=True)
+        step()
+        res_host["dq"].copy_(dq, non_blocking=True)
+        res_host["dk"].copy_(dk, non_blocking=True)
+        res_host["dv"].copy_(dv, non_blocking=True)
+    x1.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = x0.elapsed_time(x1)
+    if world > 1:
+        t = torch.tensor([ms_e2e], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_e2e = float(t.item())
+    e2e_value = world * step_flops * n_e2e / (ms_e2e * 1e-3) / 1e12
+
+    # roofline of the dominant kernel group (timed inside the long step loop: sustained peak)
+    stages = {"bwd": (t_bwd, w.bwd_flops(), "lvx_attn_bwd (preprocess + main + dQ finalize)"),
+              "fwd": (t_fwd, w.fwd_flops(), "lvx_attn_fwd (block partials + merge)"),
+              "kv": (t_kv, w.kv_flops(), "lvx_kv_recompute")}
+    dom = max(stages, key=lambda s: stages[s][0])
+    t_dom, f_dom, dom_desc = stages[dom]
+    achieved = f_dom / (t_dom * 1e-3) / 1e12
+    tr = TRAFFIC.get(dom)
+    traffic = tr["bytes"] if tr and _file_sha(tr["source"]) == tr["sha"] else None
+    launches_per_step = 7   # kv recompute (1 tensor-core, or 2 CUDA-core), fwd partials, merge,
+    # bwd preprocess, bwd main, dQ finalize
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": a.steps,
+        "warmup": warm, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded Gaussian, shapes of the "
+        "pages' Llama-3-V cross-attention workload)",
+        "config": _config(w, world),
+        "pct_of_peak": 100.0 * value / peaks["bf16_sust"],
+        "stages_ms": {"kv_recompute": t_kv, "fwd": t_fwd, "bwd": t_bwd},
+        "stage_tflops": {s: (stages[s][1] / (stages[s][0] * 1e-3) / 1e12 if stages[s][0] else None)
+                         for s in stages},
+        "roofline": {"bound": "tensor", "kernel": dom_desc, "achieved": achieved,
+                     "peak": peaks["bf16_sust"], "unit": "TFLOP/s",
+                     "frac": achieved / peaks["bf16_sust"], "traffic": traffic,
+                     "peak_source": f"{peaks['src']} (sustained cuBLAS bf16, MEASURED_PEAKS.json)"},
+        "merge": {"ms": t_merge, "achieved_gbs": merge_gbs, "peak_gbs": peaks["hbm"],
+                  "frac": merge_gbs / peaks["hbm"], "bytes": merge_bytes},
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": n_e2e},
+        "gpu_launches": launches_per_step * a.steps,
+        "clocks": clk,
+    }
+    if world == 1 and rank == 0 and not a.no_cpu_baseline:
+        cv, cs, cores, desc = oracle_sample(w)
+        line["cpu_baseline"] = {"value": cv, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                                "sample": desc, "seconds": cs}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="lvx", choices=["lvx", "reference"])
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    a = ap.parse_args()
+    if a.impl == "reference":
+        run_reference(a)
+    else:
+        run_gpu(a)
+
+
+if __name__ == "__main__":
+    main()

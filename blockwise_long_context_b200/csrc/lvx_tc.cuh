@@ -1,0 +1,25 @@
+// Tensor-core (tcgen05 + TMA) kernels for sm_100a: entry points used by the
+// C ABI layer.
+#pragma once
+
+#include "lvx_common.cuh"
+
+namespace lvx {
+
+// Forward partials / final output with tcgen05 MMAs (bf16 inputs, d in {64, 128}).
+bool tc_fwd_supported(const Problem& p);
+cudaError_t launch_fwd_tc(const Problem& p, const void* q, const void* k, const void* v,
+                          void* out, float* lse, float* o_parts, float* l_parts, cudaStream_t s);
+
+// Backward (dK, dV written; dQ accumulated unscaled into dq_acc).
+bool tc_bwd_supported(const Problem& p);
+cudaError_t launch_bwd_tc(const Problem& p, const void* q, const void* k, const void* v,
+                          const void* dout, const float* lse, const float* D, float* dq_acc,
+                          void* dk, void* dv, cudaStream_t s);
+
+// K = y W_k and V = y W_v in one launch (bf16, fp32 accumulation).
+bool tc_gemm_supported(int M, int K, int N);
+cudaError_t launch_kv_gemm_tc(const void* y, const void* w_k, const void* w_v, void* k, void* v,
+                              int M, int K, int N, cudaStream_t s);
+
+}  // namespace lvx

@@ -1,0 +1,179 @@
+/*
+ * lvx.h — C ABI of liblvx.so: exact blockwise attention with online-softmax
+ * merging on one NVIDIA B200 (sm_100a).
+ *
+ * What is computed.  For every batch b, query head h and query row r, with
+ * key/value head g = h / (H / H_kv) and scale s (1/sqrt(d) by default):
+ *     O[b,r,h,:] = sum_j softmax_j(s * q_r . k_j) v_j,
+ *     LSE[b,h,r] = ln sum_j exp(s * q_r . k_j)            (natural log)
+ * over the visible keys j (all keys, or j <= r when causal).  This is the
+ * exact attention of "Ring Attention with Blockwise Transformers for
+ * Near-Infinite Context" (citation hub page, abstract), evaluated the way
+ * "LV-XAttn: Distributed Cross-Attention for Long Visual Inputs in
+ * Multimodal Large Language Models" (review page, "The reading", "What
+ * carries the argument", Figure 3 / Algorithm 1) evaluates it: the key/value
+ * sequence is cut into n stationary blocks, each block yields a partial
+ * output O_i and log-sum-exp statistic L_i, and the partials are combined by
+ * FlashAttention-style rescaling.  On one GPU the n blocks are processed in
+ * parallel instead of around a ring; no inter-GPU communication is involved.
+ *
+ * Layouts (all contiguous, row-major, element type set by lvx_dtype):
+ *   q, out, dout, dq : [B, S_Q,  H,    d]
+ *   k, v, dk, dv     : [B, S_KV, H_kv, d]
+ *   lse              : [B, H, S_Q]  float32, natural log
+ *   y                : [B, S_KV, d_embed];  w_k, w_v : [d_embed, H_kv*d]
+ *
+ * Ownership and ordering.  The caller owns every buffer (inputs, outputs,
+ * workspace); all pointers are device pointers unless stated otherwise.  The
+ * library never allocates or frees memory and never synchronises, except
+ * lvx_last_device_error.  Every call is enqueued on the given stream and
+ * returns before the GPU work finishes.  The library keeps no per-call state
+ * and may be called from several host threads.
+ *
+ * Errors.  Invalid arguments are reported synchronously and nothing is
+ * launched.  Launch failures return LVX_ERR_CUDA.  Kernels never trap: a
+ * bounded wait that expires inside a kernel records an error word on the
+ * device, the kernel returns, and lvx_last_device_error reports it as
+ * LVX_ERR_DEVICE_TIMEOUT.
+ */
+#ifndef LVX_H_
+#define LVX_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  LVX_OK = 0,
+  LVX_ERR_INVALID_ARG = 1,    /* null/misaligned pointer, bad size, short workspace */
+  LVX_ERR_UNSUPPORTED = 2,    /* valid but not implemented (see each call)        */
+  LVX_ERR_WORKSPACE = 3,      /* workspace smaller than the size query returned    */
+  LVX_ERR_CUDA = 4,           /* a CUDA runtime/driver call or launch failed       */
+  LVX_ERR_DEVICE_TIMEOUT = 5  /* a bounded in-kernel wait expired                  */
+} lvx_status;
+
+typedef enum { LVX_FP32 = 0, LVX_BF16 = 1 } lvx_dtype;
+
+/* A cudaStream_t passed as an opaque pointer; NULL is the legacy default stream. */
+typedef void* lvx_stream;
+
+/* Returns a static, human-readable name for a status code. */
+const char* lvx_status_string(lvx_status s);
+
+/* Library version as 10000*major + 100*minor + patch. */
+int lvx_version(void);
+
+/*
+ * Workspace bytes that lvx_attn_fwd needs for these arguments (0 when
+ * n_blocks == 1).  Layout, each part starting on a 256-byte boundary:
+ *   O_parts [n_blocks, B, H, S_Q, d] float32   normalised partial outputs O_i
+ *   L_parts [n_blocks, B, H, S_Q]    float32   partial log-sum-exp L_i
+ * For causal calls only the partials of blocks j <= (block of row r) are
+ * written; the others are left untouched.  Returns 0 for invalid shapes.
+ */
+size_t lvx_attn_fwd_workspace(int B, int H, int H_kv, int S_Q, int S_KV, int d,
+                              int n_blocks, int causal, lvx_dtype dt);
+
+/*
+ * Blockwise attention forward.
+ *   LV-XAttn review page, Figure 3 / Algorithm 1: key/value block i of n
+ *   (keys [i*ceil(S_KV/n), min((i+1)*ceil(S_KV/n), S_KV))) produces the
+ *   partial (O_i, L_i) of attention over that block alone; "What carries the
+ *   argument": the partials are combined by rescaling,
+ *     L = M + ln sum_i exp(L_i - M),  M = max_i L_i;   O = sum_i exp(L_i - L) O_i.
+ *   An empty block contributes the identity (O_i, L_i) = (0, -inf).
+ * Causal (self-attention only, S_Q == S_KV): key j is visible to query r iff
+ *   j <= r; query rows use the same n-block partition, block pairs
+ *   (query block i, key block j) with j > i are skipped, and within the
+ *   diagonal pair tiles entirely above the diagonal are skipped.
+ * Arguments:
+ *   q, k, v     inputs (device, dtype dt); out [B,S_Q,H,d] (device, dtype dt);
+ *   lse         [B,H,S_Q] float32 output (device); may not be NULL.
+ *   scale       softmax scale; <= 0 selects 1/sqrt(d).
+ *   workspace   device buffer of at least lvx_attn_fwd_workspace(...) bytes,
+ *               or NULL when that size is 0.
+ * Constraints (else LVX_ERR_INVALID_ARG): all sizes >= 1, H % H_kv == 0,
+ *   1 <= n_blocks <= S_KV, pointers 16-byte aligned, ws_bytes large enough.
+ * LVX_ERR_UNSUPPORTED: d > 128 or d % 8 != 0; causal with S_Q != S_KV;
+ *   unknown dtype.
+ * bf16 with d in {64, 128} runs the tcgen05 tensor-core kernel; fp32 (and
+ *   bf16 with other d) runs an fp32 CUDA-core kernel.  Accumulation and the
+ *   softmax statistics are fp32 in both.
+ */
+lvx_status lvx_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
+                        int B, int H, int H_kv, int S_Q, int S_KV, int d,
+                        int n_blocks, int causal, lvx_dtype dt, float scale,
+                        void* workspace, size_t ws_bytes, lvx_stream stream);
+
+/*
+ * Merge of block partials on its own (the rescaling step of lvx_attn_fwd),
+ * for callers that produce the partials elsewhere, e.g. one block per GPU.
+ *   O_parts [n, B, H, S_Q, d] float32, L_parts [n, B, H, S_Q] float32 (device)
+ *   -> out [B, S_Q, H, d] (dtype dt), lse [B, H, S_Q] float32.
+ * A row whose partials are all -inf gets out = 0 and lse = -inf.
+ * Same pointer/size rules as lvx_attn_fwd; d <= 128, d % 8 == 0.
+ */
+lvx_status lvx_merge_partials(const float* O_parts, const float* L_parts, void* out, float* lse,
+                              int n, int B, int H, int S_Q, int d, lvx_dtype dt,
+                              lvx_stream stream);
+
+/*
+ * Workspace bytes for lvx_attn_bwd.  Layout (256-byte aligned parts):
+ *   D      [B, H, S_Q]      float32  rowsum(dO o O)
+ *   dQ_acc [B, S_Q, H, d]   float32  unscaled dQ accumulator
+ */
+size_t lvx_attn_bwd_workspace(int B, int H, int H_kv, int S_Q, int S_KV, int d,
+                              int causal, lvx_dtype dt);
+
+/*
+ * Blockwise attention backward: dQ, dK, dV from the stored LSE.
+ *   The pages leave the backward pass unspecified (LV-XAttn review page,
+ *   referee report, major comment 1); this is the exact gradient of the
+ *   forward above.  P is recomputed as exp(s * q.k - LSE) from the forward's
+ *   merged lse, then
+ *     dV = P^T dO,  dP = dO V^T,  D = rowsum(dO o O),  dS = P o (dP - D),
+ *     dQ = s dS K,  dK = s dS^T Q,
+ *   with dK, dV summed over the query heads of each key/value group.
+ * Arguments: q, k, v, out, dout (dtype dt), lse (float32) are the forward's
+ *   inputs/outputs and the output gradient; dq [B,S_Q,H,d] and dk, dv
+ *   [B,S_KV,H_kv,d] (dtype dt) are overwritten.  Same constraints and
+ *   errors as lvx_attn_fwd.
+ */
+lvx_status lvx_attn_bwd(const void* q, const void* k, const void* v, const void* out,
+                        const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                        int B, int H, int H_kv, int S_Q, int S_KV, int d, int causal,
+                        lvx_dtype dt, float scale, void* workspace, size_t ws_bytes,
+                        lvx_stream stream);
+
+/*
+ * Key/value recomputation from the shared visual features.
+ *   LV-XAttn review page, "What carries the argument" and Figure 6: one copy
+ *   of y serves every cross-attention layer, and K, V are regenerated from it
+ *   when needed:  K = y W_k,  V = y W_v  (no bias).
+ *   y [B, S_KV, d_embed]; w_k, w_v [d_embed, H_kv*d] row-major; k, v outputs
+ *   [B, S_KV, H_kv, d] (= [B, S_KV, H_kv*d]).  fp32 accumulation; bf16 outputs
+ *   are rounded to nearest even.
+ * Constraints: sizes >= 1, pointers 16-byte aligned.  bf16 requires
+ *   d_embed % 64 == 0 and (H_kv*d) % 128 == 0 (tensor-core tiles); otherwise,
+ *   and for fp32, a CUDA-core kernel runs.
+ */
+lvx_status lvx_kv_recompute(const void* y, const void* w_k, const void* w_v, void* k, void* v,
+                            int B, int S_KV, int d_embed, int H_kv, int d, lvx_dtype dt,
+                            lvx_stream stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the device error word of the
+ * current device.  Returns LVX_ERR_DEVICE_TIMEOUT if any kernel since the last
+ * call gave up on a bounded wait, LVX_ERR_CUDA if the stream reported an
+ * error, LVX_OK otherwise.
+ */
+lvx_status lvx_last_device_error(lvx_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LVX_H_ */

@@ -35,5 +35,6 @@ from .attention import (  # noqa: F401
     merge_partials,
     attention_bwd,
     attention_bwd_keys,
+    attention_bwd_rows,
     kv_recompute,
 )

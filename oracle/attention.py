@@ -218,16 +218,43 @@ def attention_bwd(q, k, v, do, scale: Optional[float] = None, causal: bool = Fal
     return dq, dk, dv
 
 
+def attention_bwd_rows(q, k, v, do, rows: Sequence[int], scale: Optional[float] = None,
+                       causal: bool = False, batches: Optional[Iterable[int]] = None):
+    """dQ of ``attention_bwd`` for some query rows (all query heads).
+
+    dQ_r depends only on row r's own softmax: dQ_r = s sum_j P_rj (dP_rj - D_r) k_j.
+    Returns dq of shape [B_sel, len(rows), H, d].
+    """
+    q = _f64(q); k = _f64(k); v = _f64(v); do = _f64(do)
+    B, S_Q, H, d = q.shape
+    H_kv = k.shape[2]
+    sc = _default_scale(d, scale)
+    rows = np.asarray(rows, dtype=np.int64)
+    batches = list(range(B)) if batches is None else list(batches)
+    dq = np.zeros((len(batches), len(rows), H, d))
+    for bi, b in enumerate(batches):
+        for h in range(H):
+            g = _kv_head(h, H, H_kv)
+            P = attention_probs(q, k, scale=sc, causal=causal, b=b, h=h, rows=rows)
+            dP = do[b, rows, h, :] @ v[b, :, g, :].T
+            D = (P * dP).sum(axis=1, keepdims=True)
+            dq[bi, :, h, :] = sc * ((P * (dP - D)) @ k[b, :, g, :])
+    return dq
+
+
 def attention_bwd_keys(q, k, v, do, keys: Sequence[int], kv_heads: Iterable[int],
                        scale: Optional[float] = None, causal: bool = False,
                        batches: Optional[Iterable[int]] = None,
-                       row_chunk: int = 256):
+                       row_chunk: int = 256, rows: Optional[Sequence[int]] = None):
     """dK and dV of ``attention_bwd`` restricted to some keys and KV heads.
 
     Same definition as ``attention_bwd``; each query row's P and D need that
     row's full set of logits, so rows are evaluated independently (in chunks
     of ``row_chunk`` rows to bound memory) and only the requested key columns
-    of dK, dV are kept.  Returns dk, dv of shape [B_sel, len(keys), len(kv_heads), d].
+    of dK, dV are kept.  ``rows`` limits the query rows summed over; it is
+    only exact when the other rows give the keys no gradient (causal masking
+    with keys j > every omitted row).  Returns dk, dv of shape
+    [B_sel, len(keys), len(kv_heads), d].
     """
     q = _f64(q); k = _f64(k); v = _f64(v); do = _f64(do)
     B, S_Q, H, d = q.shape
@@ -237,21 +264,22 @@ def attention_bwd_keys(q, k, v, do, keys: Sequence[int], kv_heads: Iterable[int]
     kv_heads = list(kv_heads)
     batches = list(range(B)) if batches is None else list(batches)
     grp = H // H_kv
+    all_rows = np.arange(S_Q) if rows is None else np.asarray(rows, dtype=np.int64)
     dk = np.zeros((len(batches), len(keys), len(kv_heads), d))
     dv = np.zeros_like(dk)
     for bi, b in enumerate(batches):
         for gi, g in enumerate(kv_heads):
             for h in range(g * grp, (g + 1) * grp):
-                for r0 in range(0, S_Q, row_chunk):
-                    rows = np.arange(r0, min(r0 + row_chunk, S_Q))
-                    P = attention_probs(q, k, scale=sc, causal=causal, b=b, h=h, rows=rows)
-                    dO = do[b, rows, h, :]
+                for r0 in range(0, len(all_rows), row_chunk):
+                    rows_c = all_rows[r0:r0 + row_chunk]
+                    P = attention_probs(q, k, scale=sc, causal=causal, b=b, h=h, rows=rows_c)
+                    dO = do[b, rows_c, h, :]
                     dP = dO @ v[b, :, g, :].T
                     D = (P * dP).sum(axis=1, keepdims=True)
                     Pj = P[:, keys]
                     dSj = Pj * (dP[:, keys] - D)
                     dv[bi, :, gi, :] += Pj.T @ dO
-                    dk[bi, :, gi, :] += sc * (dSj.T @ q[b, rows, h, :])
+                    dk[bi, :, gi, :] += sc * (dSj.T @ q[b, rows_c, h, :])
     return dk, dv
 
 

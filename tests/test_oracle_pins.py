@@ -258,6 +258,26 @@ def test_bwd_keys_matches_full_backward():
     np.testing.assert_allclose(dvs, dv[:, [3, 20]], atol=1e-13)
 
 
+def test_bwd_rows_matches_full_backward():
+    for causal, (S_Q, S_KV) in ((False, (9, 21)), (True, (21, 21))):
+        q, k, v = _qkv(S_Q=S_Q, S_KV=S_KV)
+        do = _rand(q.shape, 43)
+        dq, dk, dv = oracle.attention_bwd(q, k, v, do, causal=causal)
+        rows = [0, 5, S_Q - 1]
+        np.testing.assert_allclose(oracle.attention_bwd_rows(q, k, v, do, rows, causal=causal),
+                                   dq[:, rows], atol=1e-13)
+
+
+def test_bwd_keys_tail_rows_exact_under_causal_mask():
+    q, k, v = _qkv(S_Q=40, S_KV=40)
+    do = _rand(q.shape, 44)
+    dq, dk, dv = oracle.attention_bwd(q, k, v, do, causal=True)
+    keys = np.arange(30, 40)
+    dks, dvs = oracle.attention_bwd_keys(q, k, v, do, keys, [0, 1], causal=True, rows=np.arange(30, 40))
+    np.testing.assert_allclose(dks, dk[:, keys], atol=1e-13)
+    np.testing.assert_allclose(dvs, dv[:, keys], atol=1e-13)
+
+
 # ---------------------------------------------------------------- library cross-check
 
 @pytest.mark.parametrize("causal,H,H_kv,S_Q,S_KV", [(False, 4, 2, 5, 13), (True, 4, 4, 9, 9), (False, 6, 1, 3, 7)])

@@ -1,0 +1,103 @@
+"""Backward parity: dQ, dK, dV from the CUDA path against the fp64 oracle.
+
+The GPU backward recomputes P from its own forward's log-sum-exp; the
+oracle computes the textbook gradient from its own fp64 forward.  Small
+cases compare every element; full-size workloads compare dQ on sampled rows
+and dK, dV on sampled keys of one key/value head (the oracle evaluates each
+query row's full softmax to get them), plus the gradient invariants
+sum_j dV_j = sum_r dO_r (per group) and sum_j dK_j = 0, which hold for any
+size.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from blockwise_long_context_b200 import inputs
+from blockwise_long_context_b200 import binding as lvx
+from tests._parity import compare, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+SMALL = [
+    # name,            B, H, H_kv, d,  S_Q, S_KV, causal, dtype
+    ("bf16_d128_gqa",    1, 4, 2,  128, 300, 1000, False, "bf16"),
+    ("bf16_d64",         2, 2, 2,   64, 257,  777, False, "bf16"),
+    ("bf16_causal",      1, 2, 2,  128, 700,  700, True,  "bf16"),
+    ("bf16_causal_d64",  1, 4, 1,   64, 333,  333, True,  "bf16"),
+    ("bf16_tiny",        1, 1, 1,  128,   1,    1, False, "bf16"),
+    ("bf16_d96_simt",    1, 2, 1,   96, 100,  300, False, "bf16"),
+    ("f32_small",        1, 2, 1,   64, 128,  256, False, "f32"),
+    ("f32_causal",       1, 1, 1,   32,  70,   70, True,  "f32"),
+]
+
+
+def _workload(B, H, H_kv, d, S_Q, S_KV, causal, dtype):
+    base = inputs.WORKLOADS["C0" if dtype == "f32" else "C2"]
+    return base.scaled(B=B, H=H, H_kv=H_kv, d=d, S_Q=S_Q, S_KV=S_KV, causal=causal, dtype=dtype,
+                       n_blocks=1 if S_KV < 8 else 4, backward=True, d_embed=0)
+
+
+def _run(w, host):
+    dev = {k: t.cuda() for k, t in host.items()}
+    out, lse = lvx.attention_forward(dev["q"], dev["k"], dev["v"], w.n_blocks, w.causal)
+    dq, dk, dv = lvx.attention_backward(dev["q"], dev["k"], dev["v"], out, lse, dev["do"], w.causal)
+    lvx.lvx_last_device_error()
+    torch.cuda.synchronize()
+    return out, lse, dq, dk, dv
+
+
+def _invariants(w, host, dk, dv, tol=1e-2):
+    grp = w.H // w.H_kv
+    do = host["do"].double().numpy()
+    want_dv = do.reshape(w.B, w.S_Q, w.H_kv, grp, w.d).sum(axis=(1, 3))
+    got_dv = dv.double().cpu().numpy().sum(axis=1)
+    rel = np.linalg.norm(got_dv - want_dv) / np.linalg.norm(want_dv)
+    assert rel <= tol, f"sum_j dV_j != sum_r dO_r: rel {rel:.2e}"
+    dk64 = dk.double().cpu().numpy()
+    scale = np.linalg.norm(np.abs(dk64).sum(axis=1))
+    rel_k = np.linalg.norm(dk64.sum(axis=1)) / scale
+    assert rel_k <= tol, f"sum_j dK_j != 0: {rel_k:.2e}"
+
+
+@pytest.mark.parametrize("case", SMALL, ids=[c[0] for c in SMALL])
+def test_backward_small(case):
+    name, *shape = case
+    w = _workload(*shape)
+    host = inputs.make(w, tensors=("q", "k", "v", "do"))
+    out, lse, dq, dk, dv = _run(w, host)
+    q, k, v, do = (host[t].double().numpy() for t in ("q", "k", "v", "do"))
+    dq_r, dk_r, dv_r = oracle.attention_bwd(q, k, v, do, causal=w.causal)
+    compare(dq, dq_r, w.dtype, f"{name}: dQ")
+    compare(dk, dk_r, w.dtype, f"{name}: dK")
+    compare(dv, dv_r, w.dtype, f"{name}: dV")
+    _invariants(w, host, dk, dv, tol=1e-2 if w.dtype == "bf16" else 1e-5)
+
+
+@pytest.mark.parametrize("cfg", ["C2", "C4", "C3"])
+def test_backward_full_size_sampled(cfg):
+    w = inputs.WORKLOADS[cfg]
+    host = inputs.make(w, tensors=("q", "k", "v", "do"))
+    out, lse, dq, dk, dv = _run(w, host)
+    for t in (dq, dk, dv):
+        assert torch.isfinite(t.float()).all()
+    q, k, v, do = (host[t].double().numpy() for t in ("q", "k", "v", "do"))
+    # dQ on sampled rows of every head: needs only those rows' softmax
+    rows = sample_rows(w.S_Q, w.n_blocks, count=96 if cfg == "C3" else 128)
+    B0 = 0
+    dq_ref = oracle.attention_bwd_rows(q, k, v, do, rows, causal=w.causal, batches=[B0])[0]
+    compare(dq[B0, rows], dq_ref, "bf16", f"{cfg}: dQ (sampled rows)")
+    # dK, dV on sampled keys of KV head 0, summed over all query rows of its group
+    if cfg == "C3":
+        # causal tail keys j >= S-256 get gradient only from rows r >= S-256
+        keys = np.arange(w.S_KV - 256, w.S_KV)
+        dk_r, dv_r = oracle.attention_bwd_keys(q, k, v, do, keys, [0], causal=True, batches=[B0],
+                                               rows=np.arange(w.S_Q - 256, w.S_Q))
+    else:
+        keys = sample_rows(w.S_KV, w.n_blocks, count=384, seed=1)
+        dk_r, dv_r = oracle.attention_bwd_keys(q, k, v, do, keys, [0], causal=w.causal,
+                                               batches=[B0])
+    compare(dk[B0, keys, 0], dk_r[0, :, 0], "bf16", f"{cfg}: dK (sampled keys)")
+    compare(dv[B0, keys, 0], dv_r[0, :, 0], "bf16", f"{cfg}: dV (sampled keys)")
+    _invariants(w, host, dk, dv)
