@@ -1,0 +1,459 @@
+// Backward pass on the tcgen05 tensor cores (bf16, head width 64 or 128).
+//
+// The pages leave the backward pass open (LV-XAttn review page, referee
+// report, major comment 1: the gradient of the exact formula is the check).
+// This kernel computes that exact gradient from the forward's stored
+// log-sum-exp: P = exp(s q.k - LSE), dV = P^T dO, dP = dO V^T,
+// dS = P o (dP - D) with D = rowsum(dO o O), dQ = s dS K, dK = s dS^T Q.
+//
+// One CTA owns 128 keys of one (batch, key/value head) and keeps K and V in
+// shared memory; it sweeps every 128-row query tile of every query head of
+// the group (only tiles on or below the diagonal when causal).  Per tile:
+//   S^T  = K Q^T        (SS)  -> TMEM [0,128)
+//   dP^T = V dO^T       (SS)  -> TMEM [128,256)
+//   elementwise warps: P^T = exp2(S^T * s*log2e - LSE*log2e) -> bf16 back
+//       into TMEM [0,32) and [64,96); dS^T = P^T o (dP^T - D) -> bf16 into shared memory
+//   dV  += P^T dO       (TS, A = P^T from TMEM)  -> TMEM [256,256+D)
+//   dK  += dS^T Q       (SS, dS^T read K-major)  -> TMEM [256+D,256+2D)
+//   dQ_t = dS K         (SS, the same dS^T buffer read MN-major) -> TMEM [128,128+D)
+//   the elementwise warps read dQ_t out of TMEM, release it, and add it to
+//   the fp32 dQ accumulator with vector reductions.
+// dK and dV stay in TMEM for the whole sweep (the group's query heads are
+// summed in place) and are written once at the end.
+#include "lvx_ptx.cuh"
+#include "lvx_tc.cuh"
+
+namespace lvx {
+namespace {
+
+constexpr int BKEY = 128;
+constexpr int BROW = 128;
+constexpr int kThreads = 384;
+constexpr uint32_t CHUNK = 128 * 128;   // 128 rows x 64 bf16, 128-byte swizzle
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int D>
+struct BwdLayout {
+  static constexpr uint32_t TILE = 128 * D * 2;
+  static constexpr uint32_t OFF_K = 0;
+  static constexpr uint32_t OFF_V = OFF_K + TILE;
+  static constexpr uint32_t OFF_Q = OFF_V + TILE;          // 2 stages
+  static constexpr uint32_t OFF_DO = OFF_Q + 2 * TILE;     // 2 stages
+  static constexpr uint32_t OFF_DS = OFF_DO + 2 * TILE;    // 128 keys x 128 rows bf16
+  static constexpr uint32_t OFF_LSE = OFF_DS + 2 * CHUNK;  // 2 stages x 128 fp32
+  static constexpr uint32_t OFF_DD = OFF_LSE + 2 * 512;    // 2 stages x 128 fp32
+  static constexpr uint32_t OFF_BAR = OFF_DD + 2 * 512;
+  static constexpr uint32_t USED = OFF_BAR + 256;
+  static constexpr uint32_t SLACK = 768;                   // for aligning the base to 1 KiB
+  static constexpr uint32_t BYTES = (USED + SLACK) > 118784 ? (USED + SLACK) : 118784;
+  static constexpr uint32_t IDESC_SS_KK = ptx::idesc_bf16_f32(128, 128, false, false);
+  static constexpr uint32_t IDESC_DV = ptx::idesc_bf16_f32(128, D, false, true);
+  static constexpr uint32_t IDESC_DK = ptx::idesc_bf16_f32(128, D, false, true);
+  static constexpr uint32_t IDESC_DQ = ptx::idesc_bf16_f32(128, D, true, true);
+};
+
+struct BwdArgs {
+  Problem p;
+  float* dq_acc;
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+  unsigned int* err;
+  int n_kt;   // key tiles per (batch, kv head)
+  int n_qt;   // query tiles per head
+};
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
+               "f"(c), "f"(d)
+               : "memory");
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+              const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_do,
+              const __grid_constant__ CUtensorMap map_lse, const __grid_constant__ CUtensorMap map_dd,
+              const BwdArgs a) {
+  using L = BwdLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  uint64_t* kv_full = bars + 0;
+  uint64_t* q_full = bars + 1;      // [2]
+  uint64_t* q_empty = bars + 3;     // [2]
+  uint64_t* s_full = bars + 5;
+  uint64_t* dp_full = bars + 6;
+  uint64_t* p_ready = bars + 7;
+  uint64_t* ds_ready = bars + 8;
+  uint64_t* dv_done = bars + 9;
+  uint64_t* dq_full = bars + 10;
+  uint64_t* dq_free = bars + 11;
+  uint64_t* mma_drain = bars + 12;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  if ((uint32_t)(smem - smem_raw) + L::USED > L::BYTES) {   // dynamic smem base not 1 KiB aligned
+    if (threadIdx.x == 0) record_error(a.err, kErrSmemAlign);
+    return;
+  }
+  const Problem& p = a.p;
+  const int kt = blockIdx.x % a.n_kt;
+  const int bg = blockIdx.x / a.n_kt;
+  const int g = bg % p.H_kv, b = bg / p.H_kv;
+  const int grp = p.H / p.H_kv;
+  const int n0 = kt * BKEY;
+  const int m_start = p.causal ? kt : 0;   // query tiles below the diagonal see none of these keys
+  const int per_head = a.n_qt - m_start;
+  const int I = per_head > 0 ? grp * per_head : 0;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(kv_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      ptx::mbar_init(&q_full[s], 1);
+      ptx::mbar_init(&q_empty[s], 1);
+    }
+    ptx::mbar_init(s_full, 1);
+    ptx::mbar_init(dp_full, 1);
+    ptx::mbar_init(p_ready, 256);
+    ptx::mbar_init(ds_ready, 256);
+    ptx::mbar_init(dv_done, 1);
+    ptx::mbar_init(dq_full, 1);
+    ptx::mbar_init(dq_free, 256);
+    ptx::mbar_init(mma_drain, 1);
+    *abort_flag = 0;
+    ptx::fence_barrier_init();
+  }
+  if (warp == 2) {
+    ptx::tmem_alloc(tmem_slot, 512);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS = tmem, tdP = tmem + 128, tdV = tmem + 256, tdK = tmem + 256 + D;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------------------- producer
+      ptx::tma_prefetch_desc(&map_q);
+      ptx::tma_prefetch_desc(&map_do);
+      ptx::mbar_arrive_expect_tx(kv_full, 2 * L::TILE);
+      for (int c = 0; c < D / 64; ++c) {
+        ptx::tma_load_4d(smem + L::OFF_K + c * CHUNK, &map_k, kv_full, 64 * c, g, n0, b);
+        ptx::tma_load_4d(smem + L::OFF_V + c * CHUNK, &map_v, kv_full, 64 * c, g, n0, b);
+      }
+      int issued = 0;
+      for (int i = 0; i < I; ++i) {
+        const int s = i & 1;
+        const int h = g * grp + i / per_head;
+        const int m = m_start + i % per_head;
+        if (!ptx::mbar_wait(&q_empty[s], ((i >> 1) & 1) ^ 1, a.err, kErrTimeoutTma, abort_flag)) break;
+        ptx::mbar_arrive_expect_tx(&q_full[s], 2 * L::TILE + 2 * 512);
+        for (int c = 0; c < D / 64; ++c) {
+          ptx::tma_load_4d(smem + L::OFF_Q + s * L::TILE + c * CHUNK, &map_q, &q_full[s], 64 * c, h,
+                           BROW * m, b);
+          ptx::tma_load_4d(smem + L::OFF_DO + s * L::TILE + c * CHUNK, &map_do, &q_full[s], 64 * c,
+                           h, BROW * m, b);
+        }
+        ptx::tma_load_2d(smem + L::OFF_LSE + s * 512, &map_lse, &q_full[s], BROW * m, b * p.H + h);
+        ptx::tma_load_2d(smem + L::OFF_DD + s * 512, &map_dd, &q_full[s], BROW * m, b * p.H + h);
+        issued = i + 1;
+      }
+      if (*abort_flag) {
+        ptx::mbar_wait(kv_full, 0, a.err, kErrTimeoutTma, nullptr);
+        for (int i = issued > 2 ? issued - 2 : 0; i < issued; ++i)
+          ptx::mbar_wait(&q_full[i & 1], (i >> 1) & 1, a.err, kErrTimeoutTma, nullptr);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------------------------------------------------------- MMA issuer
+      const uint32_t k_base = ptx::smem_u32(smem + L::OFF_K);
+      const uint32_t v_base = ptx::smem_u32(smem + L::OFF_V);
+      const uint32_t q_base = ptx::smem_u32(smem + L::OFF_Q);
+      const uint32_t do_base = ptx::smem_u32(smem + L::OFF_DO);
+      const uint32_t ds_base = ptx::smem_u32(smem + L::OFF_DS);
+      bool ok = ptx::mbar_wait(kv_full, 0, a.err, kErrTimeoutMma, abort_flag);
+      for (int i = 0; i < I && ok; ++i) {
+        const int s = i & 1;
+        ok = ptx::mbar_wait(&q_full[s], (i >> 1) & 1, a.err, kErrTimeoutMma, abort_flag);
+        if (ok && i > 0) ok = ptx::mbar_wait(dv_done, (i - 1) & 1, a.err, kErrTimeoutMma, abort_flag);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        const uint32_t qs = q_base + s * L::TILE, dos = do_base + s * L::TILE;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {   // S^T = K Q^T
+          const uint32_t off = (kk >> 2) * CHUNK + (kk & 3) * 32;
+          ptx::mma_ss(tS, ptx::smem_desc_sw128(k_base + off, 16, 1024),
+                      ptx::smem_desc_sw128(qs + off, 16, 1024), L::IDESC_SS_KK, kk > 0);
+        }
+        ptx::mma_commit(s_full);
+        if (i > 0) {
+          ok = ptx::mbar_wait(dq_free, (i - 1) & 1, a.err, kErrTimeoutMma, abort_flag);
+          if (!ok) break;
+          ptx::tc_fence_after();
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {   // dP^T = V dO^T
+          const uint32_t off = (kk >> 2) * CHUNK + (kk & 3) * 32;
+          ptx::mma_ss(tdP, ptx::smem_desc_sw128(v_base + off, 16, 1024),
+                      ptx::smem_desc_sw128(dos + off, 16, 1024), L::IDESC_SS_KK, kk > 0);
+        }
+        ptx::mma_commit(dp_full);
+        ok = ptx::mbar_wait(p_ready, i & 1, a.err, kErrTimeoutMma, abort_flag);
+        if (!ok) break;
+        ptx::tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < BROW / 16; ++kk)   // dV += P^T dO (P^T halves at columns 0 and 64)
+          ptx::mma_ts(tdV, tS + (kk >> 2) * 64 + (kk & 3) * 8,
+                      ptx::smem_desc_sw128(dos + kk * 2048, CHUNK, 1024),
+                      L::IDESC_DV, (i > 0 || kk > 0) ? 1u : 0u);
+        ptx::mma_commit(dv_done);
+        ok = ptx::mbar_wait(ds_ready, i & 1, a.err, kErrTimeoutMma, abort_flag);
+        if (!ok) break;
+        ptx::tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < BROW / 16; ++kk) {   // dK += dS^T Q
+          const uint32_t off = (kk >> 2) * CHUNK + (kk & 3) * 32;
+          ptx::mma_ss(tdK, ptx::smem_desc_sw128(ds_base + off, 16, 1024),
+                      ptx::smem_desc_sw128(qs + kk * 2048, CHUNK, 1024), L::IDESC_DK,
+                      (i > 0 || kk > 0) ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < BKEY / 16; ++kk)   // dQ_t = dS K
+          ptx::mma_ss(tdP, ptx::smem_desc_sw128(ds_base + kk * 2048, CHUNK, 1024),
+                      ptx::smem_desc_sw128(k_base + kk * 2048, CHUNK, 1024), L::IDESC_DQ, kk > 0);
+        ptx::mma_commit(dq_full);
+        ptx::mma_commit(&q_empty[s]);
+      }
+      ptx::mma_commit(mma_drain);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------------ elementwise
+    const int quarter = warp & 3;
+    const int hf = (warp - 4) >> 2;            // which half of the 128 query rows
+    const int j = quarter * 32 + lane;         // key within the tile (TMEM lane)
+    const int key = n0 + j;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const float sl2 = p.scale_log2;
+    uint8_t* ds_smem = smem + L::OFF_DS + hf * CHUNK + j * 128;
+    bool ok = true;
+    for (int i = 0; i < I; ++i) {
+      const int s = i & 1;
+      const int h = g * grp + i / per_head;
+      const int m = m_start + i % per_head;
+      const int r0 = BROW * m + 64 * hf;       // first query row handled by this thread
+      const float* lse_s = reinterpret_cast<const float*>(smem + L::OFF_LSE + s * 512) + 64 * hf;
+      const float* dd_s = reinterpret_cast<const float*>(smem + L::OFF_DD + s * 512) + 64 * hf;
+      // this stage's LSE and D rows (TMA) are read directly below; the stage is
+      // only refilled after the MMAs of this tile, which wait for this thread
+      ok = ptx::mbar_wait(&q_full[s], (i >> 1) & 1, a.err, kErrTimeoutSoftmax, abort_flag);
+      ok = ok && ptx::mbar_wait(s_full, i & 1, a.err, kErrTimeoutSoftmax, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      ptx::tc_fence_after();
+      float P[64];
+      {
+        uint32_t sr[64];
+        ptx::tmem_ld32(tS + lane_off + 64 * hf, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+        ptx::tmem_ld32(tS + lane_off + 64 * hf + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+        ptx::tmem_wait_ld();
+        const bool key_ok = key < p.S_KV;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const int r = r0 + c;
+          const bool vis = key_ok && r < p.S_Q && (!p.causal || key <= r);
+          P[c] = vis ? ex2(fmaf(__uint_as_float(sr[c]), sl2, -lse_s[c] * kLog2e)) : 0.f;
+        }
+      }
+      {
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) pk[c] = ptx::pack_bf16x2(P[2 * c], P[2 * c + 1]);
+        // P^T of rows [64hf, 64hf+64) goes to columns [64hf, 64hf+32): only over
+        // S^T columns this thread has already read
+        ptx::tmem_st32(tS + lane_off + 64 * hf, pk);
+        ptx::tmem_wait_st();
+      }
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(p_ready);
+      ok = ptx::mbar_wait(dp_full, i & 1, a.err, kErrTimeoutSoftmax, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      ptx::tc_fence_after();
+      {
+        uint32_t dr[64];
+        ptx::tmem_ld32(tdP + lane_off + 64 * hf, *reinterpret_cast<uint32_t(*)[32]>(&dr[0]));
+        ptx::tmem_ld32(tdP + lane_off + 64 * hf + 32, *reinterpret_cast<uint32_t(*)[32]>(&dr[32]));
+        ptx::tmem_wait_ld();
+        // dS^T row of key j, query rows r0 .. r0+63: one 128-byte swizzled row
+#pragma unroll
+        for (int c8 = 0; c8 < 8; ++c8) {
+          uint4 u;
+          u.x = ptx::pack_bf16x2(P[8 * c8 + 0] * (__uint_as_float(dr[8 * c8 + 0]) - dd_s[8 * c8 + 0]),
+                                 P[8 * c8 + 1] * (__uint_as_float(dr[8 * c8 + 1]) - dd_s[8 * c8 + 1]));
+          u.y = ptx::pack_bf16x2(P[8 * c8 + 2] * (__uint_as_float(dr[8 * c8 + 2]) - dd_s[8 * c8 + 2]),
+                                 P[8 * c8 + 3] * (__uint_as_float(dr[8 * c8 + 3]) - dd_s[8 * c8 + 3]));
+          u.z = ptx::pack_bf16x2(P[8 * c8 + 4] * (__uint_as_float(dr[8 * c8 + 4]) - dd_s[8 * c8 + 4]),
+                                 P[8 * c8 + 5] * (__uint_as_float(dr[8 * c8 + 5]) - dd_s[8 * c8 + 5]));
+          u.w = ptx::pack_bf16x2(P[8 * c8 + 6] * (__uint_as_float(dr[8 * c8 + 6]) - dd_s[8 * c8 + 6]),
+                                 P[8 * c8 + 7] * (__uint_as_float(dr[8 * c8 + 7]) - dd_s[8 * c8 + 7]));
+          *reinterpret_cast<uint4*>(ds_smem + ((c8 ^ (j & 7)) << 4)) = u;
+        }
+      }
+      ptx::fence_proxy_async_smem();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(ds_ready);
+      // dQ tile: TMEM lanes are query rows here
+      ok = ptx::mbar_wait(dq_full, i & 1, a.err, kErrTimeoutSoftmax, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      ptx::tc_fence_after();
+      {
+        constexpr int HALF = D / 2;
+        uint32_t qr[HALF];
+#pragma unroll
+        for (int c = 0; c < HALF / 32; ++c)
+          ptx::tmem_ld32(tdP + lane_off + HALF * hf + 32 * c,
+                         *reinterpret_cast<uint32_t(*)[32]>(&qr[32 * c]));
+        ptx::tmem_wait_ld();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(dq_free);
+        const int row = BROW * m + quarter * 32 + lane;
+        if (row < p.S_Q) {
+          float* dst = a.dq_acc + (((size_t)b * p.S_Q + row) * p.H + h) * D + HALF * hf;
+#pragma unroll
+          for (int c = 0; c < HALF / 4; ++c)
+            red_add_v4(dst + 4 * c, __uint_as_float(qr[4 * c]), __uint_as_float(qr[4 * c + 1]),
+                       __uint_as_float(qr[4 * c + 2]), __uint_as_float(qr[4 * c + 3]));
+        }
+      }
+    }
+    // ---------------------------------------------------------------- epilogue: dK, dV
+    if (ok && I > 0) {
+      // the last dq_full of the sweep follows the last dK and dV MMAs
+      ok = __all_sync(0xffffffffu, !*abort_flag);
+    }
+    const bool write = key < p.S_KV;
+    const size_t off = (((size_t)b * p.S_KV + key) * p.H_kv + g) * D;
+    constexpr int HALF = D / 2;
+#pragma unroll 1
+    for (int which = 0; which < 2; ++which) {
+      const uint32_t tacc = (which == 0 ? tdV : tdK) + lane_off + HALF * hf;
+      const float mul = which == 0 ? 1.f : p.scale;
+      __nv_bfloat16* out = (which == 0 ? a.dv : a.dk) + off + HALF * hf;
+#pragma unroll 1
+      for (int c = 0; c < HALF / 32; ++c) {
+        uint32_t r[32];
+        if (ok && I > 0) {
+          ptx::tmem_ld32(tacc + 32 * c, r);
+          ptx::tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) r[e] = 0u;
+        }
+        if (write && ok) {
+          uint4* dst = reinterpret_cast<uint4*>(out + 32 * c);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint4 u;
+            u.x = ptx::pack_bf16x2(__uint_as_float(r[8 * q + 0]) * mul, __uint_as_float(r[8 * q + 1]) * mul);
+            u.y = ptx::pack_bf16x2(__uint_as_float(r[8 * q + 2]) * mul, __uint_as_float(r[8 * q + 3]) * mul);
+            u.z = ptx::pack_bf16x2(__uint_as_float(r[8 * q + 4]) * mul, __uint_as_float(r[8 * q + 5]) * mul);
+            u.w = ptx::pack_bf16x2(__uint_as_float(r[8 * q + 6]) * mul, __uint_as_float(r[8 * q + 7]) * mul);
+            dst[q] = u;
+          }
+        }
+      }
+    }
+  }
+
+  // ------------------------------------------------------------------ teardown
+  __syncwarp();
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    ptx::mbar_wait(mma_drain, 0, a.err, kErrTimeoutEpilogue, nullptr);
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D>
+cudaError_t launch(const Problem& p, const void* q, const void* k, const void* v,
+                   const void* dout, const float* lse, const float* Dv, float* dq_acc, void* dk,
+                   void* dv, cudaStream_t s) {
+  using L = BwdLayout<D>;
+  CUtensorMap mq, mk, mv, mdo, mlse, mdd;
+  const uint32_t box[4] = {64, 1, 128, 1};
+  {
+    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)p.H, (uint64_t)p.S_Q, (uint64_t)p.B};
+    const uint64_t str[3] = {(uint64_t)D * 2, (uint64_t)p.H * D * 2, (uint64_t)p.S_Q * p.H * D * 2};
+    if (!encode_tensor_map(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, q, dims, str, box,
+                           CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_tensor_map(&mdo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, dout, dims, str, box,
+                           CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  }
+  {
+    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)p.H_kv, (uint64_t)p.S_KV, (uint64_t)p.B};
+    const uint64_t str[3] = {(uint64_t)D * 2, (uint64_t)p.H_kv * D * 2,
+                             (uint64_t)p.S_KV * p.H_kv * D * 2};
+    if (!encode_tensor_map(&mk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, k, dims, str, box,
+                           CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_tensor_map(&mv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, v, dims, str, box,
+                           CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  }
+  {
+    // LSE and D: [B*H, S_Q] fp32 rows; S_Q * 4 bytes must be a multiple of 16
+    const uint64_t dims[2] = {(uint64_t)p.S_Q, (uint64_t)p.B * p.H};
+    const uint64_t str[1] = {(uint64_t)p.S_Q * 4};
+    const uint32_t box2[2] = {128, 1};
+    if (!encode_tensor_map(&mlse, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, lse, dims, str, box2,
+                           CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !encode_tensor_map(&mdd, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, Dv, dims, str, box2,
+                           CU_TENSOR_MAP_SWIZZLE_NONE))
+      return cudaErrorInvalidValue;
+  }
+  BwdArgs a;
+  a.p = p;
+  a.dq_acc = dq_acc;
+  a.dk = reinterpret_cast<__nv_bfloat16*>(dk);
+  a.dv = reinterpret_cast<__nv_bfloat16*>(dv);
+  a.err = device_error_word();
+  a.n_kt = (p.S_KV + BKEY - 1) / BKEY;
+  a.n_qt = (p.S_Q + BROW - 1) / BROW;
+  if (!a.err) return cudaErrorInvalidValue;
+  const long long grid = (long long)a.n_kt * p.H_kv * p.B;
+  if (grid > 0x7fffffffll) return cudaErrorInvalidConfiguration;
+  cudaError_t e = cudaFuncSetAttribute(bwd_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       L::BYTES);
+  if (e != cudaSuccess) return e;
+  bwd_tc_kernel<D><<<(unsigned)grid, kThreads, L::BYTES, s>>>(mq, mk, mv, mdo, mlse, mdd, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+// The LSE/D rows are fetched with TMA, whose row stride must be a multiple of 16 bytes.
+bool tc_bwd_supported(const Problem& p) { return (p.d == 64 || p.d == 128) && p.S_Q % 4 == 0; }
+
+cudaError_t launch_bwd_tc(const Problem& p, const void* q, const void* k, const void* v,
+                          const void* dout, const float* lse, const float* D, float* dq_acc,
+                          void* dk, void* dv, cudaStream_t s) {
+  if (p.d == 128) return launch<128>(p, q, k, v, dout, lse, D, dq_acc, dk, dv, s);
+  if (p.d == 64) return launch<64>(p, q, k, v, dout, lse, D, dq_acc, dk, dv, s);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace lvx

@@ -30,6 +30,7 @@ enum : unsigned int {
   kErrTimeoutMma = 2,
   kErrTimeoutSoftmax = 3,
   kErrTimeoutEpilogue = 4,
+  kErrSmemAlign = 5,
 };
 
 __device__ __forceinline__ void record_error(unsigned int* word, unsigned int code) {

@@ -1,0 +1,408 @@
+// Forward block partials on the tcgen05 tensor cores (bf16 inputs, fp32
+// accumulation and softmax statistics, head width 64 or 128).
+//
+// What one CTA computes: for 256 query rows (two 128-row tiles) of one
+// (batch, head) and one stationary key/value block i, the block's partial
+// output O_i and log-sum-exp L_i (LV-XAttn review page, Figure 3 /
+// Algorithm 1: each KV block produces (O_i, L_i) for the queries it sees;
+// Ring Attention citation hub page, abstract: exact blockwise attention).
+// Inside the block the 128-key tiles are folded in with an online softmax;
+// the running maximum is only moved when it grows by more than 2^8 (the
+// exponentials stay below 256, so the deferred rescaling is exact).
+//
+// Roles (12 warps):
+//   warp 0      TMA producer: Q tiles once, K and V tiles through 2-stage rings
+//   warp 1      MMA issuer:   S_t = Q_t K^T (SS form) and O_t += P_t V (TS form,
+//                             P read from TMEM)
+//   warp 2      TMEM allocator (512 columns)
+//   warps 4-7   softmax for Q tile 0, warps 8-11 for Q tile 1: one thread per
+//               row reads S from TMEM, writes P (bf16) back over S, rescales O
+//               when needed, and finally normalises O and writes the partial.
+// TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,256+D), O_1 [256+D,256+2D).
+// A new S_t is only issued after the previous P_t V MMA completed (P_t lives
+// in S_t's columns), and O_t is only rescaled between two P_t V MMAs.
+#include "lvx_ptx.cuh"
+#include "lvx_tc.cuh"
+
+namespace lvx {
+namespace {
+
+constexpr int BQ = 128;           // query rows per tile (MMA M)
+constexpr int BKV = 128;          // keys per tile
+constexpr int NQT = 2;            // query tiles per CTA
+constexpr int KV_STAGES = 2;
+constexpr int kThreads = 384;
+constexpr uint32_t CHUNK = 128 * 128;   // one TMA box: 128 rows x 64 bf16 (128 B), swizzled
+constexpr float kRescaleThreshold = 8.0f;   // log2 units
+constexpr float kLn2 = 0.6931471805599453f;
+
+template <int D>
+struct FwdLayout {
+  static constexpr uint32_t TILE = 128 * D * 2;   // Q, K or V tile
+  static constexpr uint32_t OFF_Q = 0;
+  static constexpr uint32_t OFF_K = OFF_Q + NQT * TILE;
+  static constexpr uint32_t OFF_V = OFF_K + KV_STAGES * TILE;
+  static constexpr uint32_t OFF_BAR = OFF_V + KV_STAGES * TILE;
+  static constexpr uint32_t USED = OFF_BAR + 256 + 1024;
+  // at least ~116 KiB so that one CTA (and its 512 TMEM columns) owns the SM
+  static constexpr uint32_t BYTES = USED > 118784 ? USED : 118784;
+  static constexpr uint32_t IDESC_QK = ptx::idesc_bf16_f32(128, 128, false, false);
+  static constexpr uint32_t IDESC_PV = ptx::idesc_bf16_f32(128, D, false, true);
+};
+
+struct FwdArgs {
+  Problem p;
+  __nv_bfloat16* out;   // final output (n_blocks == 1)
+  float* lse;
+  float* o_parts;       // partials (n_blocks > 1)
+  float* l_parts;
+  unsigned int* err;
+  int n_qp;             // query tile pairs per (batch, head)
+};
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+              const __grid_constant__ CUtensorMap map_v, const FwdArgs a) {
+  using L = FwdLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  uint64_t* q_full = bars + 0;
+  uint64_t* k_full = bars + 1;
+  uint64_t* k_empty = bars + 3;
+  uint64_t* v_full = bars + 5;
+  uint64_t* v_empty = bars + 7;
+  uint64_t* s_full = bars + 9;
+  uint64_t* p_full = bars + 11;
+  uint64_t* o_done = bars + 13;
+  uint64_t* mma_drain = bars + 15;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const Problem& p = a.p;
+  int idx = blockIdx.x;
+  const int qp = idx % a.n_qp;
+  idx /= a.n_qp;
+  const int h = idx % p.H;
+  idx /= p.H;
+  const int blk = idx % p.n_blocks;
+  const int b = idx / p.n_blocks;
+  const int g = h / (p.H / p.H_kv);
+  const int m0 = qp * (NQT * BQ);
+  const int kb0 = min(blk * p.block_len, p.S_KV);
+  const int kb1 = min(kb0 + p.block_len, p.S_KV);
+  int kend = kb1;
+  if (p.causal) {
+    const int last_row = min(m0 + NQT * BQ, p.S_Q) - 1;
+    if (blk > last_row / p.block_len) return;   // block pair skipped: no row of this CTA needs it
+    kend = min(kend, last_row + 1);
+  }
+  const int T = kend > kb0 ? (kend - kb0 + BKV - 1) / BKV : 0;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(q_full, 1);
+    for (int s = 0; s < KV_STAGES; ++s) {
+      ptx::mbar_init(&k_full[s], 1);
+      ptx::mbar_init(&k_empty[s], 1);
+      ptx::mbar_init(&v_full[s], 1);
+      ptx::mbar_init(&v_empty[s], 1);
+    }
+    for (int t = 0; t < NQT; ++t) {
+      ptx::mbar_init(&s_full[t], 1);
+      ptx::mbar_init(&p_full[t], 128);
+      ptx::mbar_init(&o_done[t], 1);
+    }
+    ptx::mbar_init(mma_drain, 1);
+    *abort_flag = 0;
+    ptx::fence_barrier_init();
+  }
+  if (warp == 2) {
+    ptx::tmem_alloc(tmem_slot, 512);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0 && T > 0) {
+      // ---------------------------------------------------------------- producer
+      ptx::tma_prefetch_desc(&map_q);
+      ptx::tma_prefetch_desc(&map_k);
+      ptx::tma_prefetch_desc(&map_v);
+      ptx::mbar_arrive_expect_tx(q_full, NQT * L::TILE);
+      for (int t = 0; t < NQT; ++t)
+        for (int c = 0; c < D / 64; ++c)
+          ptx::tma_load_4d(smem + L::OFF_Q + t * L::TILE + c * CHUNK, &map_q, q_full, 64 * c, h,
+                           m0 + BQ * t, b);
+      int issued_k = 0, issued_v = 0;
+      for (int j = 0; j < T; ++j) {
+        const int s = j & 1;
+        const uint32_t ph = ((j >> 1) & 1) ^ 1;
+        const int key0 = kb0 + BKV * j;
+        if (!ptx::mbar_wait(&k_empty[s], ph, a.err, kErrTimeoutTma, abort_flag)) break;
+        ptx::mbar_arrive_expect_tx(&k_full[s], L::TILE);
+        for (int c = 0; c < D / 64; ++c)
+          ptx::tma_load_4d(smem + L::OFF_K + s * L::TILE + c * CHUNK, &map_k, &k_full[s], 64 * c,
+                           g, key0, b);
+        issued_k = j + 1;
+        if (!ptx::mbar_wait(&v_empty[s], ph, a.err, kErrTimeoutTma, abort_flag)) break;
+        ptx::mbar_arrive_expect_tx(&v_full[s], L::TILE);
+        for (int c = 0; c < D / 64; ++c)
+          ptx::tma_load_4d(smem + L::OFF_V + s * L::TILE + c * CHUNK, &map_v, &v_full[s], 64 * c,
+                           g, key0, b);
+        issued_v = j + 1;
+      }
+      if (*abort_flag) {
+        // the copies already issued must land before shared memory is released
+        ptx::mbar_wait(q_full, 0, a.err, kErrTimeoutTma, nullptr);
+        for (int j = issued_k > KV_STAGES ? issued_k - KV_STAGES : 0; j < issued_k; ++j)
+          ptx::mbar_wait(&k_full[j & 1], (j >> 1) & 1, a.err, kErrTimeoutTma, nullptr);
+        for (int j = issued_v > KV_STAGES ? issued_v - KV_STAGES : 0; j < issued_v; ++j)
+          ptx::mbar_wait(&v_full[j & 1], (j >> 1) & 1, a.err, kErrTimeoutTma, nullptr);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------------------------------------------------------- MMA issuer
+      if (T > 0 && ptx::mbar_wait(q_full, 0, a.err, kErrTimeoutMma, abort_flag)) {
+        const uint32_t q_base = ptx::smem_u32(smem + L::OFF_Q);
+        const uint32_t k_base = ptx::smem_u32(smem + L::OFF_K);
+        const uint32_t v_base = ptx::smem_u32(smem + L::OFF_V);
+        for (int j = 0; j < T; ++j) {
+          const int s = j & 1;
+          const uint32_t ph = (j >> 1) & 1;
+          if (!ptx::mbar_wait(&k_full[s], ph, a.err, kErrTimeoutMma, abort_flag)) break;
+          ptx::tc_fence_after();
+          bool ok = true;
+          for (int t = 0; t < NQT && ok; ++t) {
+            if (j > 0) {
+              ok = ptx::mbar_wait(&o_done[t], (j - 1) & 1, a.err, kErrTimeoutMma, abort_flag);
+              ptx::tc_fence_after();
+            }
+            if (!ok) break;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * CHUNK + (kk & 3) * 32;
+              const uint64_t da = ptx::smem_desc_sw128(q_base + t * L::TILE + off, 16, 1024);
+              const uint64_t db = ptx::smem_desc_sw128(k_base + s * L::TILE + off, 16, 1024);
+              ptx::mma_ss(tmem + t * 128, da, db, L::IDESC_QK, kk > 0 ? 1u : 0u);
+            }
+            ptx::mma_commit(&s_full[t]);
+          }
+          if (!ok) break;
+          ptx::mma_commit(&k_empty[s]);
+          if (!ptx::mbar_wait(&v_full[s], ph, a.err, kErrTimeoutMma, abort_flag)) break;
+          for (int t = 0; t < NQT && ok; ++t) {
+            ok = ptx::mbar_wait(&p_full[t], j & 1, a.err, kErrTimeoutMma, abort_flag);
+            if (!ok) break;
+            ptx::tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < BKV / 16; ++kk) {
+              const uint64_t db =
+                  ptx::smem_desc_sw128(v_base + s * L::TILE + kk * 16 * 128, CHUNK, 1024);
+              ptx::mma_ts(tmem + 256 + t * D, tmem + t * 128 + kk * 8, db, L::IDESC_PV,
+                          (j > 0 || kk > 0) ? 1u : 0u);
+            }
+            ptx::mma_commit(&o_done[t]);
+          }
+          if (!ok) break;
+          ptx::mma_commit(&v_empty[s]);
+        }
+      }
+      ptx::mma_commit(mma_drain);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------------ softmax
+    const int t = (warp - 4) >> 2;
+    const int quarter = warp & 3;
+    const int row_in_tile = quarter * 32 + lane;
+    const int row0_tile = m0 + BQ * t;
+    const int row = row0_tile + row_in_tile;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_off + t * 128;
+    const uint32_t tO = tmem + lane_off + 256 + t * D;
+    const float sl2 = p.scale_log2;
+    float m_ref = -INFINITY, l_sum = 0.f;
+    bool ok = true;
+    for (int j = 0; j < T; ++j) {
+      ok = ptx::mbar_wait(&s_full[t], j & 1, a.err, kErrTimeoutSoftmax, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);   // keep the warp converged for tcgen05.ld/st
+      if (!ok) break;
+      ptx::tc_fence_after();
+      uint32_t sr[128];
+      ptx::tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      ptx::tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      ptx::tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
+      ptx::tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+      ptx::tmem_wait_ld();
+      const int key0 = kb0 + BKV * j;
+      const bool need_mask = (key0 + BKV > kb1) || (p.causal && key0 + BKV - 1 > row0_tile);
+      if (need_mask) {
+        const int lim = p.causal ? min(kb1, row + 1) : kb1;   // keys [key0, lim) visible
+#pragma unroll
+        for (int i = 0; i < 128; ++i)
+          if (key0 + i >= lim) sr[i] = __float_as_uint(-INFINITY);
+      }
+      float mx = __uint_as_float(sr[0]);
+#pragma unroll
+      for (int i = 1; i < 128; ++i) mx = fmaxf(mx, __uint_as_float(sr[i]));
+      const float m_tile = mx * sl2;
+      const bool resc = m_tile > m_ref + kRescaleThreshold;
+      float alpha = 1.f;
+      if (resc) {
+        alpha = ex2(m_ref - m_tile);   // 0 when m_ref is -inf
+        m_ref = m_tile;
+        l_sum *= alpha;
+      }
+      if (j > 0 && __any_sync(0xffffffffu, resc)) {
+        // O_t is quiescent here: P_t V of tile j-1 finished before S_t of tile j was issued
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          ptx::tmem_ld32(tO + c * 32, o);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          ptx::tmem_st32(tO + c * 32, o);
+        }
+      }
+      const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float p0 = ex2(fmaf(__uint_as_float(sr[32 * c + 2 * i]), sl2, -m_use));
+          const float p1 = ex2(fmaf(__uint_as_float(sr[32 * c + 2 * i + 1]), sl2, -m_use));
+          l_sum += p0 + p1;
+          pk[i] = ptx::pack_bf16x2(p0, p1);
+        }
+        ptx::tmem_st16(tS + 16 * c, pk);
+      }
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(&p_full[t]);
+    }
+    // ---------------------------------------------------------------- epilogue
+    if (T > 0 && ok) ok = ptx::mbar_wait(&o_done[t], (T - 1) & 1, a.err, kErrTimeoutEpilogue, abort_flag);
+    ok = __all_sync(0xffffffffu, ok);
+    ptx::tc_fence_after();
+    const bool seen = T > 0 && l_sum > 0.f;
+    const float inv_l = seen ? 1.f / l_sum : 0.f;
+    const float Lrow = seen ? (m_ref + __log2f(l_sum)) * kLn2 : -INFINITY;
+    const bool write = ok && row < p.S_Q;
+    const size_t prow = (((size_t)blk * p.B + b) * p.H + h) * p.S_Q + row;
+#pragma unroll 1
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t o[32];
+      if (T > 0 && ok) {
+        ptx::tmem_ld32(tO + c * 32, o);
+        ptx::tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] = 0u;
+      }
+      if (!write) continue;
+      if (p.n_blocks == 1) {
+        uint4* dst = reinterpret_cast<uint4*>(
+            a.out + (((size_t)b * p.S_Q + row) * p.H + h) * D + c * 32);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint4 u;
+          u.x = ptx::pack_bf16x2(__uint_as_float(o[8 * q + 0]) * inv_l, __uint_as_float(o[8 * q + 1]) * inv_l);
+          u.y = ptx::pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv_l, __uint_as_float(o[8 * q + 3]) * inv_l);
+          u.z = ptx::pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv_l, __uint_as_float(o[8 * q + 5]) * inv_l);
+          u.w = ptx::pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv_l, __uint_as_float(o[8 * q + 7]) * inv_l);
+          dst[q] = u;
+        }
+      } else {
+        float4* dst = reinterpret_cast<float4*>(a.o_parts + prow * D + c * 32);
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          dst[q] = make_float4(__uint_as_float(o[4 * q + 0]) * inv_l, __uint_as_float(o[4 * q + 1]) * inv_l,
+                               __uint_as_float(o[4 * q + 2]) * inv_l, __uint_as_float(o[4 * q + 3]) * inv_l);
+      }
+    }
+    if (write) {
+      if (p.n_blocks == 1)
+        a.lse[((size_t)b * p.H + h) * p.S_Q + row] = Lrow;
+      else
+        a.l_parts[prow] = Lrow;
+    }
+  }
+
+  // ------------------------------------------------------------------ teardown
+  __syncwarp();
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    ptx::mbar_wait(mma_drain, 0, a.err, kErrTimeoutEpilogue, nullptr);
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D>
+cudaError_t launch(const Problem& p, const void* q, const void* k, const void* v, void* out,
+                   float* lse, float* o_parts, float* l_parts, cudaStream_t s) {
+  using L = FwdLayout<D>;
+  CUtensorMap mq, mk, mv;
+  const uint32_t box[4] = {64, 1, 128, 1};
+  {
+    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)p.H, (uint64_t)p.S_Q, (uint64_t)p.B};
+    const uint64_t str[3] = {(uint64_t)D * 2, (uint64_t)p.H * D * 2, (uint64_t)p.S_Q * p.H * D * 2};
+    if (!encode_tensor_map(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, q, dims, str, box,
+                           CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  }
+  {
+    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)p.H_kv, (uint64_t)p.S_KV, (uint64_t)p.B};
+    const uint64_t str[3] = {(uint64_t)D * 2, (uint64_t)p.H_kv * D * 2,
+                             (uint64_t)p.S_KV * p.H_kv * D * 2};
+    if (!encode_tensor_map(&mk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, k, dims, str, box,
+                           CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_tensor_map(&mv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, v, dims, str, box,
+                           CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  }
+  FwdArgs a;
+  a.p = p;
+  a.out = reinterpret_cast<__nv_bfloat16*>(out);
+  a.lse = lse;
+  a.o_parts = o_parts;
+  a.l_parts = l_parts;
+  a.err = device_error_word();
+  a.n_qp = (p.S_Q + NQT * BQ - 1) / (NQT * BQ);
+  if (!a.err) return cudaErrorInvalidValue;
+  const long long grid = (long long)a.n_qp * p.H * p.n_blocks * p.B;
+  if (grid > 0x7fffffffll) return cudaErrorInvalidConfiguration;
+  cudaError_t e = cudaFuncSetAttribute(fwd_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       L::BYTES);
+  if (e != cudaSuccess) return e;
+  fwd_tc_kernel<D><<<(unsigned)grid, kThreads, L::BYTES, s>>>(mq, mk, mv, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool tc_fwd_supported(const Problem& p) { return p.d == 64 || p.d == 128; }
+
+cudaError_t launch_fwd_tc(const Problem& p, const void* q, const void* k, const void* v,
+                          void* out, float* lse, float* o_parts, float* l_parts, cudaStream_t s) {
+  if (p.d == 128) return launch<128>(p, q, k, v, out, lse, o_parts, l_parts, s);
+  if (p.d == 64) return launch<64>(p, q, k, v, out, lse, o_parts, l_parts, s);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace lvx
