@@ -109,6 +109,29 @@ lvx_status lvx_attn_fwd(const void* q, const void* k, const void* v, void* out, 
                         void* workspace, size_t ws_bytes, lvx_stream stream);
 
 /*
+ * lvx_attn_fwd without a workspace, for callers that cannot allocate device
+ * memory (a runtime whose device memory is fixed at start-up, a plug-in
+ * inside a host program that owns all device allocations, a latency-critical
+ * path that must not reach an allocator).  The pages have no counterpart to
+ * this call; it computes exactly what lvx_attn_fwd computes, with the same
+ * arguments minus the workspace.
+ * The block partials live in one file-scope device array of 64 MiB
+ * (n_blocks*B*H*S_Q*d*4 + n_blocks*B*H*S_Q*4 bytes, each part rounded up to
+ * 256, must fit; otherwise LVX_ERR_WORKSPACE is returned and nothing runs).
+ * Every GPU that loads the library holds that array until the process exits.
+ * All calls on a device share it and it keeps the last call's contents;
+ * nothing in it needs to start at zero, but calls whose kernels overlap on
+ * the GPU race on it, so order them on one stream.  The first call on each
+ * device looks up the array's device address (cudaGetSymbolAddress, with that
+ * device current) and caches it; make that first call before any stream
+ * capture.  No memory is allocated or freed by this call.
+ */
+lvx_status lvx_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* out, float* lse,
+                                int B, int H, int H_kv, int S_Q, int S_KV, int d,
+                                int n_blocks, int causal, lvx_dtype dt, float scale,
+                                lvx_stream stream);
+
+/*
  * Merge of block partials on its own (the rescaling step of lvx_attn_fwd),
  * for callers that produce the partials elsewhere, e.g. one block per GPU.
  *   O_parts [n, B, H, S_Q, d] float32, L_parts [n, B, H, S_Q] float32 (device)

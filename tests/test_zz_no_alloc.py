@@ -1,0 +1,65 @@
+"""lvx_attn_fwd_noalloc: the forward pass for callers that cannot allocate.
+
+Some callers cannot hand the library a workspace: their device memory is
+fixed when they start, or a host program they are loaded into owns every
+device allocation, or their latency-critical path must not reach an
+allocator.  For them the library offers a forward entry point whose block
+partials live in one fixed 64 MiB device array inside the library.  These
+tests call it through the C ABI and check, on two calls in a row with
+different inputs (the array keeps the previous call's contents), that it
+returns what the workspace-taking entry point returns, within the bf16
+parity tolerances; and that problems too large for the array are refused
+before anything runs.  This file is collected last on purpose.
+"""
+
+import pytest
+import torch
+
+from blockwise_long_context_b200 import binding as lvx
+from blockwise_long_context_b200 import inputs
+from tests._parity import compare
+
+CASES = [
+    # B, H, H_kv, d, S_Q, S_KV, n, causal
+    (1, 4, 2, 128, 300, 2000, 4, False),
+    (1, 2, 2, 64, 513, 513, 3, True),
+]
+
+
+def _with_workspace(dev, w):
+    out = torch.empty_like(dev["q"])
+    lse = torch.empty(w.B, w.H, w.S_Q, dtype=torch.float32, device="cuda")
+    ws = lvx.fwd_workspace(dev["q"], dev["k"], w.n_blocks, w.causal)
+    lvx.lvx_attn_fwd(dev["q"], dev["k"], dev["v"], out, lse, w.n_blocks, w.causal, 0.0, ws)
+    return out, lse
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("case", CASES)
+def test_noalloc_matches_workspace_entry_point_on_two_calls(case):
+    B, H, H_kv, d, S_Q, S_KV, n, causal = case
+    base = inputs.WORKLOADS["C1"].scaled(B=B, H=H, H_kv=H_kv, d=d, S_Q=S_Q, S_KV=S_KV,
+                                         n_blocks=n, causal=causal)
+    for call in range(2):
+        # a different seed per call: the shared array still holds the previous call's partials
+        w = base.scaled(index=10 + call)
+        dev = {k: t.cuda() for k, t in inputs.make(w).items()}
+        ref_out, ref_lse = _with_workspace(dev, w)
+        out = torch.full_like(dev["q"], float("nan"))
+        lse = torch.full((B, H, S_Q), float("nan"), dtype=torch.float32, device="cuda")
+        lvx.lvx_attn_fwd_noalloc(dev["q"], dev["k"], dev["v"], out, lse, n, causal)
+        lvx.lvx_last_device_error()
+        torch.cuda.synchronize()
+        compare(out, ref_out.double().cpu().numpy(), "bf16", f"call {call}: O")
+        compare(lse, ref_lse.double().cpu().numpy(), "bf16", f"call {call}: LSE", rel_rms=1e-6)
+
+
+def test_noalloc_rejects_problems_larger_than_its_array():
+    # 8 blocks x 32 heads x 2048 rows x 129 floats = 258 MiB > 64 MiB: refused before any CUDA call
+    P16 = 16
+    st = lvx.lib().lvx_attn_fwd_noalloc(P16, P16, P16, P16, P16, 1, 32, 8, 2048, 65536, 128, 8, 0,
+                                        lvx.LVX_BF16, 0.0, None)
+    assert st == 3   # LVX_ERR_WORKSPACE
+    st = lvx.lib().lvx_attn_fwd_noalloc(None, P16, P16, P16, P16, 1, 2, 1, 4, 4, 64, 1, 0,
+                                        lvx.LVX_BF16, 0.0, None)
+    assert st == 1   # LVX_ERR_INVALID_ARG
