@@ -134,7 +134,7 @@ lvx_status lvx_merge_partials(const float* O_parts, const float* L_parts, void* 
 size_t lvx_attn_bwd_workspace(int B, int H, int H_kv, int S_Q, int S_KV, int d, int causal,
                               lvx_dtype dt) {
   if (check_shapes(B, H, H_kv, S_Q, S_KV, d, 1, causal, dt) != LVX_OK) return 0;
-  return align256((size_t)B * H * S_Q * sizeof(float)) +
+  return 2 * align256((size_t)B * H * S_Q * sizeof(float)) +
          align256((size_t)B * S_Q * H * d * sizeof(float));
 }
 
@@ -153,13 +153,14 @@ lvx_status lvx_attn_bwd(const void* q, const void* k, const void* v, const void*
   if (!(scale == scale)) return LVX_ERR_INVALID_ARG;
   const Problem p = make_problem(B, H, H_kv, S_Q, S_KV, d, 1, causal, scale);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t row_bytes = align256((size_t)B * H * S_Q * sizeof(float));
   float* D = reinterpret_cast<float*>(workspace);
-  float* dq_acc = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) +
-                                           align256((size_t)B * H * S_Q * sizeof(float)));
-  cudaError_t e = launch_bwd_pre(out, dout, D, dq_acc, B, H, S_Q, d, dt, s);
+  float* lse2 = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) + row_bytes);
+  float* dq_acc = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) + 2 * row_bytes);
+  cudaError_t e = launch_bwd_pre(out, dout, lse, D, lse2, dq_acc, B, H, S_Q, d, dt, s);
   if (e != cudaSuccess) return LVX_ERR_CUDA;
   if (dt == LVX_BF16 && tc_bwd_supported(p))
-    e = launch_bwd_tc(p, q, k, v, dout, lse, D, dq_acc, dk, dv, s);
+    e = launch_bwd_tc(p, q, k, v, dout, lse2, D, dq_acc, dk, dv, s);
   else
     e = launch_bwd_simt(p, dt, q, k, v, dout, lse, D, dq_acc, dk, dv, s);
   if (e != cudaSuccess) return LVX_ERR_CUDA;

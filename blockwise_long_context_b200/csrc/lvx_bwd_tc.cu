@@ -30,7 +30,6 @@ constexpr int BKEY = 128;
 constexpr int BROW = 128;
 constexpr int kThreads = 384;
 constexpr uint32_t CHUNK = 128 * 128;   // 128 rows x 64 bf16, 128-byte swizzle
-constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D>
 struct BwdLayout {
@@ -68,10 +67,28 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
-               "f"(c), "f"(d)
-               : "memory");
+// Adds a shared-memory tile into global memory through a tensor map (TMA
+// reduce-add in L2, asynchronous; the tile may be reused after bulk_wait_read).
+__device__ __forceinline__ void tma_reduce_add_4d(const CUtensorMap* map, const void* ssrc, int c0,
+                                                  int c1, int c2, int c3) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.4d.global.shared::cta.add.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(ptx::smem_u32(ssrc)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+// Barrier among the 8 elementwise warps only (named barrier 1).
+__device__ __forceinline__ void elementwise_sync() {
+  asm volatile("bar.sync 1, 256;" ::: "memory");
 }
 
 template <int D>
@@ -79,7 +96,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
               const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_do,
               const __grid_constant__ CUtensorMap map_lse, const __grid_constant__ CUtensorMap map_dd,
-              const BwdArgs a) {
+              const __grid_constant__ CUtensorMap map_dq, const BwdArgs a) {
   using L = BwdLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -252,6 +269,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
       const int h = g * grp + i / per_head;
       const int m = m_start + i % per_head;
       const int r0 = BROW * m + 64 * hf;       // first query row handled by this thread
+      // the LSE stage holds LSE * log2(e) (scaled by the preprocess kernel)
       const float* lse_s = reinterpret_cast<const float*>(smem + L::OFF_LSE + s * 512) + 64 * hf;
       const float* dd_s = reinterpret_cast<const float*>(smem + L::OFF_DD + s * 512) + 64 * hf;
       // this stage's LSE and D rows (TMA) are read directly below; the stage is
@@ -267,12 +285,20 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
         ptx::tmem_ld32(tS + lane_off + 64 * hf, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
         ptx::tmem_ld32(tS + lane_off + 64 * hf + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
         ptx::tmem_wait_ld();
-        const bool key_ok = key < p.S_KV;
+        // masking is needed only on the causal diagonal tile and at the ragged ends
+        const bool need_mask = (p.causal && m == kt) || (n0 + BKEY > p.S_KV) ||
+                               (BROW * m + BROW > p.S_Q);
+        if (need_mask) {
+          const bool key_ok = key < p.S_KV;
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const int r = r0 + c;
-          const bool vis = key_ok && r < p.S_Q && (!p.causal || key <= r);
-          P[c] = vis ? ex2(fmaf(__uint_as_float(sr[c]), sl2, -lse_s[c] * kLog2e)) : 0.f;
+          for (int c = 0; c < 64; ++c) {
+            const int r = r0 + c;
+            const bool vis = key_ok && r < p.S_Q && (!p.causal || key <= r);
+            P[c] = vis ? ex2(fmaf(__uint_as_float(sr[c]), sl2, -lse_s[c])) : 0.f;
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) P[c] = ex2(fmaf(__uint_as_float(sr[c]), sl2, -lse_s[c]));
         }
       }
       {
@@ -290,23 +316,25 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       ptx::tc_fence_after();
-      {
-        uint32_t dr[64];
-        ptx::tmem_ld32(tdP + lane_off + 64 * hf, *reinterpret_cast<uint32_t(*)[32]>(&dr[0]));
-        ptx::tmem_ld32(tdP + lane_off + 64 * hf + 32, *reinterpret_cast<uint32_t(*)[32]>(&dr[32]));
-        ptx::tmem_wait_ld();
-        // dS^T row of key j, query rows r0 .. r0+63: one 128-byte swizzled row
+      // dS^T row of key j, query rows r0 .. r0+63 (one 128-byte swizzled row),
+      // in two 32-column halves to bound register use
 #pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8) {
+      for (int half = 0; half < 2; ++half) {
+        uint32_t dr[32];
+        ptx::tmem_ld32(tdP + lane_off + 64 * hf + 32 * half, dr);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int q8 = 0; q8 < 4; ++q8) {
+          const int c8 = 4 * half + q8;
+          float e[8];
+#pragma unroll
+          for (int t = 0; t < 8; ++t)
+            e[t] = P[8 * c8 + t] * (__uint_as_float(dr[8 * q8 + t]) - dd_s[8 * c8 + t]);
           uint4 u;
-          u.x = ptx::pack_bf16x2(P[8 * c8 + 0] * (__uint_as_float(dr[8 * c8 + 0]) - dd_s[8 * c8 + 0]),
-                                 P[8 * c8 + 1] * (__uint_as_float(dr[8 * c8 + 1]) - dd_s[8 * c8 + 1]));
-          u.y = ptx::pack_bf16x2(P[8 * c8 + 2] * (__uint_as_float(dr[8 * c8 + 2]) - dd_s[8 * c8 + 2]),
-                                 P[8 * c8 + 3] * (__uint_as_float(dr[8 * c8 + 3]) - dd_s[8 * c8 + 3]));
-          u.z = ptx::pack_bf16x2(P[8 * c8 + 4] * (__uint_as_float(dr[8 * c8 + 4]) - dd_s[8 * c8 + 4]),
-                                 P[8 * c8 + 5] * (__uint_as_float(dr[8 * c8 + 5]) - dd_s[8 * c8 + 5]));
-          u.w = ptx::pack_bf16x2(P[8 * c8 + 6] * (__uint_as_float(dr[8 * c8 + 6]) - dd_s[8 * c8 + 6]),
-                                 P[8 * c8 + 7] * (__uint_as_float(dr[8 * c8 + 7]) - dd_s[8 * c8 + 7]));
+          u.x = ptx::pack_bf16x2(e[0], e[1]);
+          u.y = ptx::pack_bf16x2(e[2], e[3]);
+          u.z = ptx::pack_bf16x2(e[4], e[5]);
+          u.w = ptx::pack_bf16x2(e[6], e[7]);
           *reinterpret_cast<uint4*>(ds_smem + ((c8 ^ (j & 7)) << 4)) = u;
         }
       }
@@ -319,6 +347,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
       if (!ok) break;
       ptx::tc_fence_after();
       {
+        // dQ_t rows: TMEM lane = query row; this thread holds columns [HALF*hf, HALF*hf + HALF)
         constexpr int HALF = D / 2;
         uint32_t qr[HALF];
 #pragma unroll
@@ -328,16 +357,37 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
         ptx::tmem_wait_ld();
         ptx::tc_fence_before();
         ptx::mbar_arrive(dq_free);
-        const int row = BROW * m + quarter * 32 + lane;
-        if (row < p.S_Q) {
-          float* dst = a.dq_acc + (((size_t)b * p.S_Q + row) * p.H + h) * D + HALF * hf;
+        // The dS^T buffer is free here (dq_full follows the dK and dQ MMAs that read
+        // it).  Each warp stages 32 rows x 32 columns (4 KiB) of dQ_t in its own
+        // quarter of it, 128-byte swizzled, and adds the piece to dQ_acc with one
+        // TMA reduce-add; pieces outside the sequence are clipped by the TMA unit.
+        uint8_t* stage = smem + L::OFF_DS + (warp - 4) * 4096;
+        const int h_row0 = BROW * m + quarter * 32;
 #pragma unroll
-          for (int c = 0; c < HALF / 4; ++c)
-            red_add_v4(dst + 4 * c, __uint_as_float(qr[4 * c]), __uint_as_float(qr[4 * c + 1]),
-                       __uint_as_float(qr[4 * c + 2]), __uint_as_float(qr[4 * c + 3]));
+        for (int piece = 0; piece < HALF / 32; ++piece) {
+          if (piece > 0) {
+            if (lane == 0) bulk_wait_read();
+            __syncwarp();
+          }
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(stage + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+                make_uint4(qr[32 * piece + 4 * c], qr[32 * piece + 4 * c + 1],
+                           qr[32 * piece + 4 * c + 2], qr[32 * piece + 4 * c + 3]);
+          ptx::fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_reduce_add_4d(&map_dq, stage, HALF * hf + 32 * piece, h, h_row0, b);
+            bulk_commit();
+          }
         }
+        if (lane == 0) bulk_wait_read();
+        __syncwarp();
+        // nobody writes dS of the next tile over a piece another warp still stages
+        elementwise_sync();
       }
     }
+    if (lane == 0) bulk_wait_all();
     // ---------------------------------------------------------------- epilogue: dK, dV
     if (ok && I > 0) {
       // the last dq_full of the sweep follows the last dK and dV MMAs
@@ -393,7 +443,7 @@ cudaError_t launch(const Problem& p, const void* q, const void* k, const void* v
                    const void* dout, const float* lse, const float* Dv, float* dq_acc, void* dk,
                    void* dv, cudaStream_t s) {
   using L = BwdLayout<D>;
-  CUtensorMap mq, mk, mv, mdo, mlse, mdd;
+  CUtensorMap mq, mk, mv, mdo, mlse, mdd, mdq;
   const uint32_t box[4] = {64, 1, 128, 1};
   {
     const uint64_t dims[4] = {(uint64_t)D, (uint64_t)p.H, (uint64_t)p.S_Q, (uint64_t)p.B};
@@ -425,6 +475,14 @@ cudaError_t launch(const Problem& p, const void* q, const void* k, const void* v
                            CU_TENSOR_MAP_SWIZZLE_NONE))
       return cudaErrorInvalidValue;
   }
+  {
+    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)p.H, (uint64_t)p.S_Q, (uint64_t)p.B};
+    const uint64_t str[3] = {(uint64_t)D * 4, (uint64_t)p.H * D * 4, (uint64_t)p.S_Q * p.H * D * 4};
+    const uint32_t box4[4] = {32, 1, 32, 1};
+    if (!encode_tensor_map(&mdq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dq_acc, dims, str, box4,
+                           CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  }
   BwdArgs a;
   a.p = p;
   a.dq_acc = dq_acc;
@@ -439,7 +497,7 @@ cudaError_t launch(const Problem& p, const void* q, const void* k, const void* v
   cudaError_t e = cudaFuncSetAttribute(bwd_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        L::BYTES);
   if (e != cudaSuccess) return e;
-  bwd_tc_kernel<D><<<(unsigned)grid, kThreads, L::BYTES, s>>>(mq, mk, mv, mdo, mlse, mdd, a);
+  bwd_tc_kernel<D><<<(unsigned)grid, kThreads, L::BYTES, s>>>(mq, mk, mv, mdo, mlse, mdd, mdq, a);
   return cudaGetLastError();
 }
 

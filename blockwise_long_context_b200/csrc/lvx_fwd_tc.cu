@@ -66,6 +66,22 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// 2^x on the FMA pipe: x = n + f with n = round(x), |f| <= 1/2; 2^f from a
+// cubic fitted by fit_exp2.py (max relative error 7.5e-5, far below the
+// bf16 rounding P receives); n is added to the exponent field.  Adding
+// 1.5 * 2^23 leaves round(x) in the low mantissa bits of t.  x is clamped at
+// -127 so the exponent cannot wrap; callers use it only on unmasked tiles,
+// where the argument is finite.
+constexpr int kPolyEvery = 4;
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -127.f);
+  const float t = x + 12582912.f;
+  const float f = x - (t - 12582912.f);
+  const float p = fmaf(fmaf(fmaf(5.517164990e-02f, f, 2.426111400e-01f), f, 6.932609677e-01f), f,
+                       9.999280572e-01f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
@@ -175,49 +191,67 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------------------------------------------------------- MMA issuer
+      // Issue order: S0_0, S1_0, PV0_0, then per tile j >= 1
+      //   S0_j, PV1_{j-1}, S1_j, PV0_j,  and finally PV1_{T-1}.
+      // Softmax of Q tile 0 on S0_j overlaps PV1_{j-1} and S1_j on the tensor
+      // core, softmax of tile 1 overlaps PV0_j and S0_{j+1}, so the two softmax
+      // groups take turns on the exponential unit.  S_t of tile j overwrites
+      // P_t of tile j-1 right after the MMA that reads it; tcgen05.mma ops of
+      // one thread execute in issue order, so that read completes first.
       if (T > 0 && ptx::mbar_wait(q_full, 0, a.err, kErrTimeoutMma, abort_flag)) {
         const uint32_t q_base = ptx::smem_u32(smem + L::OFF_Q);
         const uint32_t k_base = ptx::smem_u32(smem + L::OFF_K);
         const uint32_t v_base = ptx::smem_u32(smem + L::OFF_V);
-        for (int j = 0; j < T; ++j) {
+        auto issue_s = [&](int t, int j) {
+          const int s = j & 1;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * CHUNK + (kk & 3) * 32;
+            const uint64_t da = ptx::smem_desc_sw128(q_base + t * L::TILE + off, 16, 1024);
+            const uint64_t db = ptx::smem_desc_sw128(k_base + s * L::TILE + off, 16, 1024);
+            ptx::mma_ss(tmem + t * 128, da, db, L::IDESC_QK, kk > 0 ? 1u : 0u);
+          }
+          ptx::mma_commit(&s_full[t]);
+        };
+        auto issue_pv = [&](int t, int j) {
+          const int s = j & 1;
+#pragma unroll
+          for (int kk = 0; kk < BKV / 16; ++kk) {
+            const uint64_t db =
+                ptx::smem_desc_sw128(v_base + s * L::TILE + kk * 16 * 128, CHUNK, 1024);
+            ptx::mma_ts(tmem + 256 + t * D, tmem + t * 128 + kk * 8, db, L::IDESC_PV,
+                        (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          ptx::mma_commit(&o_done[t]);
+        };
+        bool ok = true;
+        for (int j = 0; j < T && ok; ++j) {
           const int s = j & 1;
           const uint32_t ph = (j >> 1) & 1;
-          if (!ptx::mbar_wait(&k_full[s], ph, a.err, kErrTimeoutMma, abort_flag)) break;
-          ptx::tc_fence_after();
-          bool ok = true;
-          for (int t = 0; t < NQT && ok; ++t) {
-            if (j > 0) {
-              ok = ptx::mbar_wait(&o_done[t], (j - 1) & 1, a.err, kErrTimeoutMma, abort_flag);
-              ptx::tc_fence_after();
-            }
-            if (!ok) break;
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t off = (kk >> 2) * CHUNK + (kk & 3) * 32;
-              const uint64_t da = ptx::smem_desc_sw128(q_base + t * L::TILE + off, 16, 1024);
-              const uint64_t db = ptx::smem_desc_sw128(k_base + s * L::TILE + off, 16, 1024);
-              ptx::mma_ss(tmem + t * 128, da, db, L::IDESC_QK, kk > 0 ? 1u : 0u);
-            }
-            ptx::mma_commit(&s_full[t]);
-          }
+          ok = ptx::mbar_wait(&k_full[s], ph, a.err, kErrTimeoutMma, abort_flag);
           if (!ok) break;
-          ptx::mma_commit(&k_empty[s]);
-          if (!ptx::mbar_wait(&v_full[s], ph, a.err, kErrTimeoutMma, abort_flag)) break;
-          for (int t = 0; t < NQT && ok; ++t) {
-            ok = ptx::mbar_wait(&p_full[t], j & 1, a.err, kErrTimeoutMma, abort_flag);
+          ptx::tc_fence_after();
+          issue_s(0, j);
+          if (j > 0) {
+            // PV1 of the previous tile (its V stage is released afterwards)
+            ok = ptx::mbar_wait(&p_full[1], (j - 1) & 1, a.err, kErrTimeoutMma, abort_flag);
             if (!ok) break;
             ptx::tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < BKV / 16; ++kk) {
-              const uint64_t db =
-                  ptx::smem_desc_sw128(v_base + s * L::TILE + kk * 16 * 128, CHUNK, 1024);
-              ptx::mma_ts(tmem + 256 + t * D, tmem + t * 128 + kk * 8, db, L::IDESC_PV,
-                          (j > 0 || kk > 0) ? 1u : 0u);
-            }
-            ptx::mma_commit(&o_done[t]);
+            issue_pv(1, j - 1);
+            ptx::mma_commit(&v_empty[(j - 1) & 1]);
           }
+          issue_s(1, j);
+          ptx::mma_commit(&k_empty[s]);
+          ok = ptx::mbar_wait(&v_full[s], ph, a.err, kErrTimeoutMma, abort_flag);
+          if (ok) ok = ptx::mbar_wait(&p_full[0], j & 1, a.err, kErrTimeoutMma, abort_flag);
           if (!ok) break;
-          ptx::mma_commit(&v_empty[s]);
+          ptx::tc_fence_after();
+          issue_pv(0, j);
+        }
+        if (ok && ptx::mbar_wait(&p_full[1], (T - 1) & 1, a.err, kErrTimeoutMma, abort_flag)) {
+          ptx::tc_fence_after();
+          issue_pv(1, T - 1);
+          ptx::mma_commit(&v_empty[(T - 1) & 1]);
         }
       }
       ptx::mma_commit(mma_drain);
@@ -278,17 +312,36 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
         }
       }
       const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
+      if (need_mask) {
+        // masked tiles: every exponential on the special-function unit (exact 0 for -inf)
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16];
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float p0 = ex2(fmaf(__uint_as_float(sr[32 * c + 2 * i]), sl2, -m_use));
-          const float p1 = ex2(fmaf(__uint_as_float(sr[32 * c + 2 * i + 1]), sl2, -m_use));
-          l_sum += p0 + p1;
-          pk[i] = ptx::pack_bf16x2(p0, p1);
+          for (int i = 0; i < 16; ++i) {
+            const float p0 = ex2(fmaf(__uint_as_float(sr[32 * c + 2 * i]), sl2, -m_use));
+            const float p1 = ex2(fmaf(__uint_as_float(sr[32 * c + 2 * i + 1]), sl2, -m_use));
+            l_sum += p0 + p1;
+            pk[i] = ptx::pack_bf16x2(p0, p1);
+          }
+          ptx::tmem_st16(tS + 16 * c, pk);
         }
-        ptx::tmem_st16(tS + 16 * c, pk);
+      } else {
+        // one exponential in kPolyEvery on the FMA pipe, the rest on the SFU
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float x0 = fmaf(__uint_as_float(sr[32 * c + 2 * i]), sl2, -m_use);
+            const float x1 = fmaf(__uint_as_float(sr[32 * c + 2 * i + 1]), sl2, -m_use);
+            const float p0 = ex2(x0);
+            const float p1 = ((2 * i + 1) % kPolyEvery == kPolyEvery - 1) ? exp2_poly(x1) : ex2(x1);
+            l_sum += p0 + p1;
+            pk[i] = ptx::pack_bf16x2(p0, p1);
+          }
+          ptx::tmem_st16(tS + 16 * c, pk);
+        }
       }
       ptx::tmem_wait_st();
       ptx::tc_fence_before();

@@ -48,7 +48,7 @@ def test_workspace_sizes():
     assert lvx.lvx_attn_fwd_workspace(1, 32, 8, 2048, 65536, 128, 1, 0, lvx.LVX_BF16) == 0
     assert lvx.lvx_attn_fwd_workspace(1, 3, 2, 10, 10, 64, 2, 0, lvx.LVX_BF16) == 0   # H % H_kv
     bw = lvx.lvx_attn_bwd_workspace(1, 2, 1, 100, 300, 64, 0, lvx.LVX_BF16)
-    assert bw == 1024 + 100 * 2 * 64 * 4   # D rounded to 256 bytes, then dQ accumulator
+    assert bw == 2 * 1024 + 100 * 2 * 64 * 4   # D and LSE*log2(e), 256-byte aligned, then dQ_acc
 
 
 P16 = 16   # a non-null, 16-byte-aligned address; never dereferenced on these paths
