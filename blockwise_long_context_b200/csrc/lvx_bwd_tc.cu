@@ -16,8 +16,8 @@
 //   dV  += P^T dO       (TS, A = P^T from TMEM)  -> TMEM [256,256+D)
 //   dK  += dS^T Q       (SS, dS^T read K-major)  -> TMEM [256+D,256+2D)
 //   dQ_t = dS K         (SS, the same dS^T buffer read MN-major) -> TMEM [128,128+D)
-//   the elementwise warps read dQ_t out of TMEM, release it, and add it to
-//   the fp32 dQ accumulator with vector reductions.
+//   a drain warpgroup reads dQ_t out of TMEM, releases it, and adds it to the
+//   fp32 dQ accumulator with TMA reduce-add (staged in the dS buffer).
 // dK and dV stay in TMEM for the whole sweep (the group's query heads are
 // summed in place) and are written once at the end.
 #include "lvx_ptx.cuh"
@@ -28,7 +28,16 @@ namespace {
 
 constexpr int BKEY = 128;
 constexpr int BROW = 128;
-constexpr int kThreads = 384;
+constexpr int kThreads = 512;
+// Register split (launched at 128 per thread): warpgroup 0 (producer, MMA
+// issuer, allocator) 56, the two elementwise warpgroups 168, the dQ drain
+// warpgroup 120:  128 x 56 + 256 x 168 + 128 x 120 = 65536 = 512 x 128.
+constexpr uint32_t kRegsControl = 56;
+constexpr uint32_t kRegsElementwise = 168;
+constexpr uint32_t kRegsDrain = 120;
+static_assert(128 * kRegsControl + 256 * kRegsElementwise + 128 * kRegsDrain <=
+                  65536 / kThreads * kThreads,
+              "register split exceeds the launch allocation");
 constexpr uint32_t CHUNK = 128 * 128;   // 128 rows x 64 bf16, 128-byte swizzle
 
 template <int D>
@@ -86,10 +95,7 @@ __device__ __forceinline__ void bulk_wait_read() {
 __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
-// Barrier among the 8 elementwise warps only (named barrier 1).
-__device__ __forceinline__ void elementwise_sync() {
-  asm volatile("bar.sync 1, 256;" ::: "memory");
-}
+
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -113,7 +119,8 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
   uint64_t* dq_full = bars + 10;
   uint64_t* dq_free = bars + 11;
   uint64_t* mma_drain = bars + 12;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
+  uint64_t* stage_free = bars + 13;   // dQ staging (in the dS buffer) read back by the TMA
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   if ((uint32_t)(smem - smem_raw) + L::USED > L::BYTES) {   // dynamic smem base not 1 KiB aligned
@@ -143,8 +150,9 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
     ptx::mbar_init(ds_ready, 256);
     ptx::mbar_init(dv_done, 1);
     ptx::mbar_init(dq_full, 1);
-    ptx::mbar_init(dq_free, 256);
+    ptx::mbar_init(dq_free, 128);
     ptx::mbar_init(mma_drain, 1);
+    ptx::mbar_init(stage_free, 4);
     *abort_flag = 0;
     ptx::fence_barrier_init();
   }
@@ -158,103 +166,107 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
   const uint32_t tmem = *tmem_slot;
   const uint32_t tS = tmem, tdP = tmem + 128, tdV = tmem + 256, tdK = tmem + 256 + D;
 
-  if (warp == 0) {
-    if (lane == 0) {
-      // ---------------------------------------------------------------- producer
-      ptx::tma_prefetch_desc(&map_q);
-      ptx::tma_prefetch_desc(&map_do);
-      ptx::mbar_arrive_expect_tx(kv_full, 2 * L::TILE);
-      for (int c = 0; c < D / 64; ++c) {
-        ptx::tma_load_4d(smem + L::OFF_K + c * CHUNK, &map_k, kv_full, 64 * c, g, n0, b);
-        ptx::tma_load_4d(smem + L::OFF_V + c * CHUNK, &map_v, kv_full, 64 * c, g, n0, b);
-      }
-      int issued = 0;
-      for (int i = 0; i < I; ++i) {
-        const int s = i & 1;
-        const int h = g * grp + i / per_head;
-        const int m = m_start + i % per_head;
-        if (!ptx::mbar_wait(&q_empty[s], ((i >> 1) & 1) ^ 1, a.err, kErrTimeoutTma, abort_flag)) break;
-        ptx::mbar_arrive_expect_tx(&q_full[s], 2 * L::TILE + 2 * 512);
+  if (warp < 4) {
+    ptx::setmaxnreg_dec<kRegsControl>();
+    if (warp == 0) {
+      if (lane == 0) {
+        // ---------------------------------------------------------------- producer
+        ptx::tma_prefetch_desc(&map_q);
+        ptx::tma_prefetch_desc(&map_do);
+        ptx::mbar_arrive_expect_tx(kv_full, 2 * L::TILE);
         for (int c = 0; c < D / 64; ++c) {
-          ptx::tma_load_4d(smem + L::OFF_Q + s * L::TILE + c * CHUNK, &map_q, &q_full[s], 64 * c, h,
-                           BROW * m, b);
-          ptx::tma_load_4d(smem + L::OFF_DO + s * L::TILE + c * CHUNK, &map_do, &q_full[s], 64 * c,
-                           h, BROW * m, b);
+          ptx::tma_load_4d(smem + L::OFF_K + c * CHUNK, &map_k, kv_full, 64 * c, g, n0, b);
+          ptx::tma_load_4d(smem + L::OFF_V + c * CHUNK, &map_v, kv_full, 64 * c, g, n0, b);
         }
-        ptx::tma_load_2d(smem + L::OFF_LSE + s * 512, &map_lse, &q_full[s], BROW * m, b * p.H + h);
-        ptx::tma_load_2d(smem + L::OFF_DD + s * 512, &map_dd, &q_full[s], BROW * m, b * p.H + h);
-        issued = i + 1;
-      }
-      if (*abort_flag) {
-        ptx::mbar_wait(kv_full, 0, a.err, kErrTimeoutTma, nullptr);
-        for (int i = issued > 2 ? issued - 2 : 0; i < issued; ++i)
-          ptx::mbar_wait(&q_full[i & 1], (i >> 1) & 1, a.err, kErrTimeoutTma, nullptr);
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------------------------------------------------------- MMA issuer
-      const uint32_t k_base = ptx::smem_u32(smem + L::OFF_K);
-      const uint32_t v_base = ptx::smem_u32(smem + L::OFF_V);
-      const uint32_t q_base = ptx::smem_u32(smem + L::OFF_Q);
-      const uint32_t do_base = ptx::smem_u32(smem + L::OFF_DO);
-      const uint32_t ds_base = ptx::smem_u32(smem + L::OFF_DS);
-      bool ok = ptx::mbar_wait(kv_full, 0, a.err, kErrTimeoutMma, abort_flag);
-      for (int i = 0; i < I && ok; ++i) {
-        const int s = i & 1;
-        ok = ptx::mbar_wait(&q_full[s], (i >> 1) & 1, a.err, kErrTimeoutMma, abort_flag);
-        if (ok && i > 0) ok = ptx::mbar_wait(dv_done, (i - 1) & 1, a.err, kErrTimeoutMma, abort_flag);
-        if (!ok) break;
-        ptx::tc_fence_after();
-        const uint32_t qs = q_base + s * L::TILE, dos = do_base + s * L::TILE;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {   // S^T = K Q^T
-          const uint32_t off = (kk >> 2) * CHUNK + (kk & 3) * 32;
-          ptx::mma_ss(tS, ptx::smem_desc_sw128(k_base + off, 16, 1024),
-                      ptx::smem_desc_sw128(qs + off, 16, 1024), L::IDESC_SS_KK, kk > 0);
+        int issued = 0;
+        for (int i = 0; i < I; ++i) {
+          const int s = i & 1;
+          const int h = g * grp + i / per_head;
+          const int m = m_start + i % per_head;
+          if (!ptx::mbar_wait(&q_empty[s], ((i >> 1) & 1) ^ 1, a.err, kErrTimeoutTma, abort_flag)) break;
+          ptx::mbar_arrive_expect_tx(&q_full[s], 2 * L::TILE + 2 * 512);
+          for (int c = 0; c < D / 64; ++c) {
+            ptx::tma_load_4d(smem + L::OFF_Q + s * L::TILE + c * CHUNK, &map_q, &q_full[s], 64 * c, h,
+                             BROW * m, b);
+            ptx::tma_load_4d(smem + L::OFF_DO + s * L::TILE + c * CHUNK, &map_do, &q_full[s], 64 * c,
+                             h, BROW * m, b);
+          }
+          ptx::tma_load_2d(smem + L::OFF_LSE + s * 512, &map_lse, &q_full[s], BROW * m, b * p.H + h);
+          ptx::tma_load_2d(smem + L::OFF_DD + s * 512, &map_dd, &q_full[s], BROW * m, b * p.H + h);
+          issued = i + 1;
         }
-        ptx::mma_commit(s_full);
-        if (i > 0) {
-          ok = ptx::mbar_wait(dq_free, (i - 1) & 1, a.err, kErrTimeoutMma, abort_flag);
+        if (*abort_flag) {
+          ptx::mbar_wait(kv_full, 0, a.err, kErrTimeoutTma, nullptr);
+          for (int i = issued > 2 ? issued - 2 : 0; i < issued; ++i)
+            ptx::mbar_wait(&q_full[i & 1], (i >> 1) & 1, a.err, kErrTimeoutTma, nullptr);
+        }
+      }
+    } else if (warp == 1) {
+      if (lane == 0) {
+        // ---------------------------------------------------------------- MMA issuer
+        const uint32_t k_base = ptx::smem_u32(smem + L::OFF_K);
+        const uint32_t v_base = ptx::smem_u32(smem + L::OFF_V);
+        const uint32_t q_base = ptx::smem_u32(smem + L::OFF_Q);
+        const uint32_t do_base = ptx::smem_u32(smem + L::OFF_DO);
+        const uint32_t ds_base = ptx::smem_u32(smem + L::OFF_DS);
+        bool ok = ptx::mbar_wait(kv_full, 0, a.err, kErrTimeoutMma, abort_flag);
+        for (int i = 0; i < I && ok; ++i) {
+          const int s = i & 1;
+          ok = ptx::mbar_wait(&q_full[s], (i >> 1) & 1, a.err, kErrTimeoutMma, abort_flag);
+          if (ok && i > 0) ok = ptx::mbar_wait(dv_done, (i - 1) & 1, a.err, kErrTimeoutMma, abort_flag);
           if (!ok) break;
           ptx::tc_fence_after();
+          const uint32_t qs = q_base + s * L::TILE, dos = do_base + s * L::TILE;
+  #pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {   // S^T = K Q^T
+            const uint32_t off = (kk >> 2) * CHUNK + (kk & 3) * 32;
+            ptx::mma_ss(tS, ptx::smem_desc_sw128(k_base + off, 16, 1024),
+                        ptx::smem_desc_sw128(qs + off, 16, 1024), L::IDESC_SS_KK, kk > 0);
+          }
+          ptx::mma_commit(s_full);
+          if (i > 0) {
+            ok = ptx::mbar_wait(dq_free, (i - 1) & 1, a.err, kErrTimeoutMma, abort_flag);
+            if (!ok) break;
+            ptx::tc_fence_after();
+          }
+  #pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {   // dP^T = V dO^T
+            const uint32_t off = (kk >> 2) * CHUNK + (kk & 3) * 32;
+            ptx::mma_ss(tdP, ptx::smem_desc_sw128(v_base + off, 16, 1024),
+                        ptx::smem_desc_sw128(dos + off, 16, 1024), L::IDESC_SS_KK, kk > 0);
+          }
+          ptx::mma_commit(dp_full);
+          ok = ptx::mbar_wait(p_ready, i & 1, a.err, kErrTimeoutMma, abort_flag);
+          if (!ok) break;
+          ptx::tc_fence_after();
+  #pragma unroll
+          for (int kk = 0; kk < BROW / 16; ++kk)   // dV += P^T dO (P^T halves at columns 0 and 64)
+            ptx::mma_ts(tdV, tS + (kk >> 2) * 64 + (kk & 3) * 8,
+                        ptx::smem_desc_sw128(dos + kk * 2048, CHUNK, 1024),
+                        L::IDESC_DV, (i > 0 || kk > 0) ? 1u : 0u);
+          ptx::mma_commit(dv_done);
+          ok = ptx::mbar_wait(ds_ready, i & 1, a.err, kErrTimeoutMma, abort_flag);
+          if (!ok) break;
+          ptx::tc_fence_after();
+  #pragma unroll
+          for (int kk = 0; kk < BROW / 16; ++kk) {   // dK += dS^T Q
+            const uint32_t off = (kk >> 2) * CHUNK + (kk & 3) * 32;
+            ptx::mma_ss(tdK, ptx::smem_desc_sw128(ds_base + off, 16, 1024),
+                        ptx::smem_desc_sw128(qs + kk * 2048, CHUNK, 1024), L::IDESC_DK,
+                        (i > 0 || kk > 0) ? 1u : 0u);
+          }
+  #pragma unroll
+          for (int kk = 0; kk < BKEY / 16; ++kk)   // dQ_t = dS K
+            ptx::mma_ss(tdP, ptx::smem_desc_sw128(ds_base + kk * 2048, CHUNK, 1024),
+                        ptx::smem_desc_sw128(k_base + kk * 2048, CHUNK, 1024), L::IDESC_DQ, kk > 0);
+          ptx::mma_commit(dq_full);
+          ptx::mma_commit(&q_empty[s]);
         }
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {   // dP^T = V dO^T
-          const uint32_t off = (kk >> 2) * CHUNK + (kk & 3) * 32;
-          ptx::mma_ss(tdP, ptx::smem_desc_sw128(v_base + off, 16, 1024),
-                      ptx::smem_desc_sw128(dos + off, 16, 1024), L::IDESC_SS_KK, kk > 0);
-        }
-        ptx::mma_commit(dp_full);
-        ok = ptx::mbar_wait(p_ready, i & 1, a.err, kErrTimeoutMma, abort_flag);
-        if (!ok) break;
-        ptx::tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < BROW / 16; ++kk)   // dV += P^T dO (P^T halves at columns 0 and 64)
-          ptx::mma_ts(tdV, tS + (kk >> 2) * 64 + (kk & 3) * 8,
-                      ptx::smem_desc_sw128(dos + kk * 2048, CHUNK, 1024),
-                      L::IDESC_DV, (i > 0 || kk > 0) ? 1u : 0u);
-        ptx::mma_commit(dv_done);
-        ok = ptx::mbar_wait(ds_ready, i & 1, a.err, kErrTimeoutMma, abort_flag);
-        if (!ok) break;
-        ptx::tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < BROW / 16; ++kk) {   // dK += dS^T Q
-          const uint32_t off = (kk >> 2) * CHUNK + (kk & 3) * 32;
-          ptx::mma_ss(tdK, ptx::smem_desc_sw128(ds_base + off, 16, 1024),
-                      ptx::smem_desc_sw128(qs + kk * 2048, CHUNK, 1024), L::IDESC_DK,
-                      (i > 0 || kk > 0) ? 1u : 0u);
-        }
-#pragma unroll
-        for (int kk = 0; kk < BKEY / 16; ++kk)   // dQ_t = dS K
-          ptx::mma_ss(tdP, ptx::smem_desc_sw128(ds_base + kk * 2048, CHUNK, 1024),
-                      ptx::smem_desc_sw128(k_base + kk * 2048, CHUNK, 1024), L::IDESC_DQ, kk > 0);
-        ptx::mma_commit(dq_full);
-        ptx::mma_commit(&q_empty[s]);
+        ptx::mma_commit(mma_drain);
       }
-      ptx::mma_commit(mma_drain);
     }
-  } else if (warp >= 4) {
+  } else if (warp < 12) {
+    ptx::setmaxnreg_inc<kRegsElementwise>();
     // ------------------------------------------------------------------ elementwise
     const int quarter = warp & 3;
     const int hf = (warp - 4) >> 2;            // which half of the 128 query rows
@@ -313,6 +325,10 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
       ptx::tc_fence_before();
       ptx::mbar_arrive(p_ready);
       ok = ptx::mbar_wait(dp_full, i & 1, a.err, kErrTimeoutSoftmax, abort_flag);
+      // the dS buffer doubles as the drain's dQ staging: wait until the drain
+      // warps' TMA reductions of the previous tile have read it
+      if (ok && i > 0)
+        ok = ptx::mbar_wait(stage_free, (i - 1) & 1, a.err, kErrTimeoutSoftmax, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       ptx::tc_fence_after();
@@ -341,57 +357,13 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
       ptx::fence_proxy_async_smem();
       ptx::tc_fence_before();
       ptx::mbar_arrive(ds_ready);
-      // dQ tile: TMEM lanes are query rows here
-      ok = ptx::mbar_wait(dq_full, i & 1, a.err, kErrTimeoutSoftmax, abort_flag);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      ptx::tc_fence_after();
-      {
-        // dQ_t rows: TMEM lane = query row; this thread holds columns [HALF*hf, HALF*hf + HALF)
-        constexpr int HALF = D / 2;
-        uint32_t qr[HALF];
-#pragma unroll
-        for (int c = 0; c < HALF / 32; ++c)
-          ptx::tmem_ld32(tdP + lane_off + HALF * hf + 32 * c,
-                         *reinterpret_cast<uint32_t(*)[32]>(&qr[32 * c]));
-        ptx::tmem_wait_ld();
-        ptx::tc_fence_before();
-        ptx::mbar_arrive(dq_free);
-        // The dS^T buffer is free here (dq_full follows the dK and dQ MMAs that read
-        // it).  Each warp stages 32 rows x 32 columns (4 KiB) of dQ_t in its own
-        // quarter of it, 128-byte swizzled, and adds the piece to dQ_acc with one
-        // TMA reduce-add; pieces outside the sequence are clipped by the TMA unit.
-        uint8_t* stage = smem + L::OFF_DS + (warp - 4) * 4096;
-        const int h_row0 = BROW * m + quarter * 32;
-#pragma unroll
-        for (int piece = 0; piece < HALF / 32; ++piece) {
-          if (piece > 0) {
-            if (lane == 0) bulk_wait_read();
-            __syncwarp();
-          }
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<uint4*>(stage + lane * 128 + ((c ^ (lane & 7)) << 4)) =
-                make_uint4(qr[32 * piece + 4 * c], qr[32 * piece + 4 * c + 1],
-                           qr[32 * piece + 4 * c + 2], qr[32 * piece + 4 * c + 3]);
-          ptx::fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_reduce_add_4d(&map_dq, stage, HALF * hf + 32 * piece, h, h_row0, b);
-            bulk_commit();
-          }
-        }
-        if (lane == 0) bulk_wait_read();
-        __syncwarp();
-        // nobody writes dS of the next tile over a piece another warp still stages
-        elementwise_sync();
-      }
     }
-    if (lane == 0) bulk_wait_all();
     // ---------------------------------------------------------------- epilogue: dK, dV
     if (ok && I > 0) {
       // the last dq_full of the sweep follows the last dK and dV MMAs
-      ok = __all_sync(0xffffffffu, !*abort_flag);
+      ok = ptx::mbar_wait(dq_full, (I - 1) & 1, a.err, kErrTimeoutEpilogue, abort_flag);
+      ok = __all_sync(0xffffffffu, ok && !*abort_flag);
+      ptx::tc_fence_after();
     }
     const bool write = key < p.S_KV;
     const size_t off = (((size_t)b * p.S_KV + key) * p.H_kv + g) * D;
@@ -425,6 +397,63 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
         }
       }
     }
+  } else {
+    ptx::setmaxnreg_dec<kRegsDrain>();
+    // ------------------------------------------------------------------ dQ drain
+    // Warp 12+q reads TMEM lanes 32q..32q+31 (query rows) of dQ_t, releases the
+    // columns to the MMA warp, and adds the rows to dQ_acc: 32x32 pieces are
+    // staged 128-byte swizzled in its own 8 KiB of the dS buffer (free between
+    // the dQ MMA and the next tile's dS) and reduced with TMA reduce-add.
+    const int quarter = warp & 3;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    uint8_t* stage = smem + L::OFF_DS + quarter * 8192;
+    bool ok = true;
+    for (int i = 0; i < I; ++i) {
+      const int h = g * grp + i / per_head;
+      const int m = m_start + i % per_head;
+      const int row0 = BROW * m + quarter * 32;
+      ok = ptx::mbar_wait(dq_full, i & 1, a.err, kErrTimeoutSoftmax, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      ptx::tc_fence_after();
+#pragma unroll
+      for (int round = 0; round < D / 64; ++round) {
+        uint32_t qr[64];
+        ptx::tmem_ld32(tdP + lane_off + 64 * round, *reinterpret_cast<uint32_t(*)[32]>(&qr[0]));
+        ptx::tmem_ld32(tdP + lane_off + 64 * round + 32, *reinterpret_cast<uint32_t(*)[32]>(&qr[32]));
+        ptx::tmem_wait_ld();
+        if (round == D / 64 - 1) {
+          ptx::tc_fence_before();
+          ptx::mbar_arrive(dq_free);
+        }
+        if (round > 0) {   // the previous round's pieces must have been read by the TMA
+          if (lane == 0) bulk_wait_read();
+          __syncwarp();
+        }
+#pragma unroll
+        for (int piece = 0; piece < 2; ++piece) {
+          uint8_t* st = stage + piece * 4096;
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(st + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+                make_uint4(qr[32 * piece + 4 * c], qr[32 * piece + 4 * c + 1],
+                           qr[32 * piece + 4 * c + 2], qr[32 * piece + 4 * c + 3]);
+        }
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_reduce_add_4d(&map_dq, stage, 64 * round, h, row0, b);
+          tma_reduce_add_4d(&map_dq, stage + 4096, 64 * round + 32, h, row0, b);
+          bulk_commit();
+        }
+      }
+      if (lane == 0) {
+        bulk_wait_read();
+        ptx::mbar_arrive(stage_free);
+      }
+      __syncwarp();
+    }
+    if (lane == 0) bulk_wait_all();
   }
 
   // ------------------------------------------------------------------ teardown

@@ -32,6 +32,13 @@ constexpr int BKV = 128;          // keys per tile
 constexpr int NQT = 2;            // query tiles per CTA
 constexpr int KV_STAGES = 2;
 constexpr int kThreads = 384;
+// Register split: launched at 168 per thread (384 x 168 = 64512); warpgroup 0
+// (producer, MMA issuer, allocator) gives up 64, the two softmax warpgroups
+// take 32 each: 128 x 104 + 256 x 200 = 64512.
+constexpr uint32_t kRegsControl = 104;
+constexpr uint32_t kRegsSoftmax = 200;
+static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= 65536 / kThreads * kThreads,
+              "register split exceeds the launch allocation");
 constexpr uint32_t CHUNK = 128 * 128;   // one TMA box: 128 rows x 64 bf16 (128 B), swizzled
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
 constexpr float kLn2 = 0.6931471805599453f;
@@ -66,13 +73,38 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// Packed fp32 pairs (Blackwell FFMA2 / FADD2) and the three-input maximum.
+__device__ __forceinline__ uint64_t pk2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void upk2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // 2^x on the FMA pipe: x = n + f with n = round(x), |f| <= 1/2; 2^f from a
 // cubic fitted by fit_exp2.py (max relative error 7.5e-5, far below the
 // bf16 rounding P receives); n is added to the exponent field.  Adding
 // 1.5 * 2^23 leaves round(x) in the low mantissa bits of t.  x is clamped at
 // -127 so the exponent cannot wrap; callers use it only on unmasked tiles,
 // where the argument is finite.
-constexpr int kPolyEvery = 4;
+constexpr int kPolyEvery = 4;   // one pair of exponentials in kPolyEvery on the FMA pipe
 __device__ __forceinline__ float exp2_poly(float x) {
   x = fmaxf(x, -127.f);
   const float t = x + 12582912.f;
@@ -80,6 +112,28 @@ __device__ __forceinline__ float exp2_poly(float x) {
   const float p = fmaf(fmaf(fmaf(5.517164990e-02f, f, 2.426111400e-01f), f, 6.932609677e-01f), f,
                        9.999280572e-01f);
   return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// The same for a packed pair, with the fp32 arithmetic on FFMA2 / FADD2.
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
+  float x0, x1;
+  upk2(x2, x0, x1);
+  x2 = pk2(fmaxf(x0, -127.f), fmaxf(x1, -127.f));
+  const uint64_t magic = pk2(12582912.f, 12582912.f);
+  const uint64_t nmagic = pk2(-12582912.f, -12582912.f);
+  const uint64_t t = fadd2(x2, magic);
+  const uint64_t r = fadd2(t, nmagic);
+  float r0, r1;
+  upk2(r, r0, r1);
+  const uint64_t f = fadd2(x2, pk2(-r0, -r1));
+  uint64_t p = ffma2(pk2(5.517164990e-02f, 5.517164990e-02f), f, pk2(2.426111400e-01f, 2.426111400e-01f));
+  p = ffma2(p, f, pk2(6.932609677e-01f, 6.932609677e-01f));
+  p = ffma2(p, f, pk2(9.999280572e-01f, 9.999280572e-01f));
+  float p0, p1, t0, t1;
+  upk2(p, p0, p1);
+  upk2(t, t0, t1);
+  return pk2(__int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23)),
+             __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23)));
 }
 
 template <int D>
@@ -149,114 +203,117 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
-  if (warp == 0) {
-    if (lane == 0 && T > 0) {
-      // ---------------------------------------------------------------- producer
-      ptx::tma_prefetch_desc(&map_q);
-      ptx::tma_prefetch_desc(&map_k);
-      ptx::tma_prefetch_desc(&map_v);
-      ptx::mbar_arrive_expect_tx(q_full, NQT * L::TILE);
-      for (int t = 0; t < NQT; ++t)
-        for (int c = 0; c < D / 64; ++c)
-          ptx::tma_load_4d(smem + L::OFF_Q + t * L::TILE + c * CHUNK, &map_q, q_full, 64 * c, h,
-                           m0 + BQ * t, b);
-      int issued_k = 0, issued_v = 0;
-      for (int j = 0; j < T; ++j) {
-        const int s = j & 1;
-        const uint32_t ph = ((j >> 1) & 1) ^ 1;
-        const int key0 = kb0 + BKV * j;
-        if (!ptx::mbar_wait(&k_empty[s], ph, a.err, kErrTimeoutTma, abort_flag)) break;
-        ptx::mbar_arrive_expect_tx(&k_full[s], L::TILE);
-        for (int c = 0; c < D / 64; ++c)
-          ptx::tma_load_4d(smem + L::OFF_K + s * L::TILE + c * CHUNK, &map_k, &k_full[s], 64 * c,
-                           g, key0, b);
-        issued_k = j + 1;
-        if (!ptx::mbar_wait(&v_empty[s], ph, a.err, kErrTimeoutTma, abort_flag)) break;
-        ptx::mbar_arrive_expect_tx(&v_full[s], L::TILE);
-        for (int c = 0; c < D / 64; ++c)
-          ptx::tma_load_4d(smem + L::OFF_V + s * L::TILE + c * CHUNK, &map_v, &v_full[s], 64 * c,
-                           g, key0, b);
-        issued_v = j + 1;
+  if (warp < 4) {
+    ptx::setmaxnreg_dec<kRegsControl>();
+    if (warp == 0) {
+      if (lane == 0 && T > 0) {
+        // ---------------------------------------------------------------- producer
+        ptx::tma_prefetch_desc(&map_q);
+        ptx::tma_prefetch_desc(&map_k);
+        ptx::tma_prefetch_desc(&map_v);
+        ptx::mbar_arrive_expect_tx(q_full, NQT * L::TILE);
+        for (int t = 0; t < NQT; ++t)
+          for (int c = 0; c < D / 64; ++c)
+            ptx::tma_load_4d(smem + L::OFF_Q + t * L::TILE + c * CHUNK, &map_q, q_full, 64 * c, h,
+                             m0 + BQ * t, b);
+        int issued_k = 0, issued_v = 0;
+        for (int j = 0; j < T; ++j) {
+          const int s = j & 1;
+          const uint32_t ph = ((j >> 1) & 1) ^ 1;
+          const int key0 = kb0 + BKV * j;
+          if (!ptx::mbar_wait(&k_empty[s], ph, a.err, kErrTimeoutTma, abort_flag)) break;
+          ptx::mbar_arrive_expect_tx(&k_full[s], L::TILE);
+          for (int c = 0; c < D / 64; ++c)
+            ptx::tma_load_4d(smem + L::OFF_K + s * L::TILE + c * CHUNK, &map_k, &k_full[s], 64 * c,
+                             g, key0, b);
+          issued_k = j + 1;
+          if (!ptx::mbar_wait(&v_empty[s], ph, a.err, kErrTimeoutTma, abort_flag)) break;
+          ptx::mbar_arrive_expect_tx(&v_full[s], L::TILE);
+          for (int c = 0; c < D / 64; ++c)
+            ptx::tma_load_4d(smem + L::OFF_V + s * L::TILE + c * CHUNK, &map_v, &v_full[s], 64 * c,
+                             g, key0, b);
+          issued_v = j + 1;
+        }
+        if (*abort_flag) {
+          // the copies already issued must land before shared memory is released
+          ptx::mbar_wait(q_full, 0, a.err, kErrTimeoutTma, nullptr);
+          for (int j = issued_k > KV_STAGES ? issued_k - KV_STAGES : 0; j < issued_k; ++j)
+            ptx::mbar_wait(&k_full[j & 1], (j >> 1) & 1, a.err, kErrTimeoutTma, nullptr);
+          for (int j = issued_v > KV_STAGES ? issued_v - KV_STAGES : 0; j < issued_v; ++j)
+            ptx::mbar_wait(&v_full[j & 1], (j >> 1) & 1, a.err, kErrTimeoutTma, nullptr);
+        }
       }
-      if (*abort_flag) {
-        // the copies already issued must land before shared memory is released
-        ptx::mbar_wait(q_full, 0, a.err, kErrTimeoutTma, nullptr);
-        for (int j = issued_k > KV_STAGES ? issued_k - KV_STAGES : 0; j < issued_k; ++j)
-          ptx::mbar_wait(&k_full[j & 1], (j >> 1) & 1, a.err, kErrTimeoutTma, nullptr);
-        for (int j = issued_v > KV_STAGES ? issued_v - KV_STAGES : 0; j < issued_v; ++j)
-          ptx::mbar_wait(&v_full[j & 1], (j >> 1) & 1, a.err, kErrTimeoutTma, nullptr);
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------------------------------------------------------- MMA issuer
-      // Issue order: S0_0, S1_0, PV0_0, then per tile j >= 1
-      //   S0_j, PV1_{j-1}, S1_j, PV0_j,  and finally PV1_{T-1}.
-      // Softmax of Q tile 0 on S0_j overlaps PV1_{j-1} and S1_j on the tensor
-      // core, softmax of tile 1 overlaps PV0_j and S0_{j+1}, so the two softmax
-      // groups take turns on the exponential unit.  S_t of tile j overwrites
-      // P_t of tile j-1 right after the MMA that reads it; tcgen05.mma ops of
-      // one thread execute in issue order, so that read completes first.
-      if (T > 0 && ptx::mbar_wait(q_full, 0, a.err, kErrTimeoutMma, abort_flag)) {
-        const uint32_t q_base = ptx::smem_u32(smem + L::OFF_Q);
-        const uint32_t k_base = ptx::smem_u32(smem + L::OFF_K);
-        const uint32_t v_base = ptx::smem_u32(smem + L::OFF_V);
-        auto issue_s = [&](int t, int j) {
-          const int s = j & 1;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * CHUNK + (kk & 3) * 32;
-            const uint64_t da = ptx::smem_desc_sw128(q_base + t * L::TILE + off, 16, 1024);
-            const uint64_t db = ptx::smem_desc_sw128(k_base + s * L::TILE + off, 16, 1024);
-            ptx::mma_ss(tmem + t * 128, da, db, L::IDESC_QK, kk > 0 ? 1u : 0u);
-          }
-          ptx::mma_commit(&s_full[t]);
-        };
-        auto issue_pv = [&](int t, int j) {
-          const int s = j & 1;
-#pragma unroll
-          for (int kk = 0; kk < BKV / 16; ++kk) {
-            const uint64_t db =
-                ptx::smem_desc_sw128(v_base + s * L::TILE + kk * 16 * 128, CHUNK, 1024);
-            ptx::mma_ts(tmem + 256 + t * D, tmem + t * 128 + kk * 8, db, L::IDESC_PV,
-                        (j > 0 || kk > 0) ? 1u : 0u);
-          }
-          ptx::mma_commit(&o_done[t]);
-        };
-        bool ok = true;
-        for (int j = 0; j < T && ok; ++j) {
-          const int s = j & 1;
-          const uint32_t ph = (j >> 1) & 1;
-          ok = ptx::mbar_wait(&k_full[s], ph, a.err, kErrTimeoutMma, abort_flag);
-          if (!ok) break;
-          ptx::tc_fence_after();
-          issue_s(0, j);
-          if (j > 0) {
-            // PV1 of the previous tile (its V stage is released afterwards)
-            ok = ptx::mbar_wait(&p_full[1], (j - 1) & 1, a.err, kErrTimeoutMma, abort_flag);
+    } else if (warp == 1) {
+      if (lane == 0) {
+        // ---------------------------------------------------------------- MMA issuer
+        // Issue order: S0_0, S1_0, PV0_0, then per tile j >= 1
+        //   S0_j, PV1_{j-1}, S1_j, PV0_j,  and finally PV1_{T-1}.
+        // Softmax of Q tile 0 on S0_j overlaps PV1_{j-1} and S1_j on the tensor
+        // core, softmax of tile 1 overlaps PV0_j and S0_{j+1}, so the two softmax
+        // groups take turns on the exponential unit.  S_t of tile j overwrites
+        // P_t of tile j-1 right after the MMA that reads it; tcgen05.mma ops of
+        // one thread execute in issue order, so that read completes first.
+        if (T > 0 && ptx::mbar_wait(q_full, 0, a.err, kErrTimeoutMma, abort_flag)) {
+          const uint32_t q_base = ptx::smem_u32(smem + L::OFF_Q);
+          const uint32_t k_base = ptx::smem_u32(smem + L::OFF_K);
+          const uint32_t v_base = ptx::smem_u32(smem + L::OFF_V);
+          auto issue_s = [&](int t, int j) {
+            const int s = j & 1;
+  #pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * CHUNK + (kk & 3) * 32;
+              const uint64_t da = ptx::smem_desc_sw128(q_base + t * L::TILE + off, 16, 1024);
+              const uint64_t db = ptx::smem_desc_sw128(k_base + s * L::TILE + off, 16, 1024);
+              ptx::mma_ss(tmem + t * 128, da, db, L::IDESC_QK, kk > 0 ? 1u : 0u);
+            }
+            ptx::mma_commit(&s_full[t]);
+          };
+          auto issue_pv = [&](int t, int j) {
+            const int s = j & 1;
+  #pragma unroll
+            for (int kk = 0; kk < BKV / 16; ++kk) {
+              const uint64_t db =
+                  ptx::smem_desc_sw128(v_base + s * L::TILE + kk * 16 * 128, CHUNK, 1024);
+              ptx::mma_ts(tmem + 256 + t * D, tmem + t * 128 + kk * 8, db, L::IDESC_PV,
+                          (j > 0 || kk > 0) ? 1u : 0u);
+            }
+            ptx::mma_commit(&o_done[t]);
+          };
+          bool ok = true;
+          for (int j = 0; j < T && ok; ++j) {
+            const int s = j & 1;
+            const uint32_t ph = (j >> 1) & 1;
+            ok = ptx::mbar_wait(&k_full[s], ph, a.err, kErrTimeoutMma, abort_flag);
             if (!ok) break;
             ptx::tc_fence_after();
-            issue_pv(1, j - 1);
-            ptx::mma_commit(&v_empty[(j - 1) & 1]);
+            issue_s(0, j);
+            if (j > 0) {
+              // PV1 of the previous tile (its V stage is released afterwards)
+              ok = ptx::mbar_wait(&p_full[1], (j - 1) & 1, a.err, kErrTimeoutMma, abort_flag);
+              if (!ok) break;
+              ptx::tc_fence_after();
+              issue_pv(1, j - 1);
+              ptx::mma_commit(&v_empty[(j - 1) & 1]);
+            }
+            issue_s(1, j);
+            ptx::mma_commit(&k_empty[s]);
+            ok = ptx::mbar_wait(&v_full[s], ph, a.err, kErrTimeoutMma, abort_flag);
+            if (ok) ok = ptx::mbar_wait(&p_full[0], j & 1, a.err, kErrTimeoutMma, abort_flag);
+            if (!ok) break;
+            ptx::tc_fence_after();
+            issue_pv(0, j);
           }
-          issue_s(1, j);
-          ptx::mma_commit(&k_empty[s]);
-          ok = ptx::mbar_wait(&v_full[s], ph, a.err, kErrTimeoutMma, abort_flag);
-          if (ok) ok = ptx::mbar_wait(&p_full[0], j & 1, a.err, kErrTimeoutMma, abort_flag);
-          if (!ok) break;
-          ptx::tc_fence_after();
-          issue_pv(0, j);
+          if (ok && ptx::mbar_wait(&p_full[1], (T - 1) & 1, a.err, kErrTimeoutMma, abort_flag)) {
+            ptx::tc_fence_after();
+            issue_pv(1, T - 1);
+            ptx::mma_commit(&v_empty[(T - 1) & 1]);
+          }
         }
-        if (ok && ptx::mbar_wait(&p_full[1], (T - 1) & 1, a.err, kErrTimeoutMma, abort_flag)) {
-          ptx::tc_fence_after();
-          issue_pv(1, T - 1);
-          ptx::mma_commit(&v_empty[(T - 1) & 1]);
-        }
+        ptx::mma_commit(mma_drain);
       }
-      ptx::mma_commit(mma_drain);
     }
-  } else if (warp >= 4) {
+  } else {
+    ptx::setmaxnreg_inc<kRegsSoftmax>();
     // ------------------------------------------------------------------ softmax
     const int t = (warp - 4) >> 2;
     const int quarter = warp & 3;
@@ -290,7 +347,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
       }
       float mx = __uint_as_float(sr[0]);
 #pragma unroll
-      for (int i = 1; i < 128; ++i) mx = fmaxf(mx, __uint_as_float(sr[i]));
+      for (int i = 1; i < 127; i += 2) mx = fmax3(mx, __uint_as_float(sr[i]), __uint_as_float(sr[i + 1]));
+      mx = fmaxf(mx, __uint_as_float(sr[127]));
       const float m_tile = mx * sl2;
       const bool resc = m_tile > m_ref + kRescaleThreshold;
       float alpha = 1.f;
@@ -327,21 +385,37 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
           ptx::tmem_st16(tS + 16 * c, pk);
         }
       } else {
-        // one exponential in kPolyEvery on the FMA pipe, the rest on the SFU
+        // packed pairs: x = s*scale - m with FFMA2, one pair in kPolyEvery through the
+        // FMA-pipe polynomial and the rest on the SFU, row sum with FADD2
+        const uint64_t sl2x2 = pk2(sl2, sl2);
+        const uint64_t negm2 = pk2(-m_use, -m_use);
+        uint64_t acc2 = pk2(0.f, 0.f);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float x0 = fmaf(__uint_as_float(sr[32 * c + 2 * i]), sl2, -m_use);
-            const float x1 = fmaf(__uint_as_float(sr[32 * c + 2 * i + 1]), sl2, -m_use);
-            const float p0 = ex2(x0);
-            const float p1 = ((2 * i + 1) % kPolyEvery == kPolyEvery - 1) ? exp2_poly(x1) : ex2(x1);
-            l_sum += p0 + p1;
+            const uint64_t s2 = pk2(__uint_as_float(sr[32 * c + 2 * i]),
+                                    __uint_as_float(sr[32 * c + 2 * i + 1]));
+            const uint64_t x2 = ffma2(s2, sl2x2, negm2);
+            uint64_t e2;
+            if (i % kPolyEvery == kPolyEvery - 1) {
+              e2 = exp2_poly2(x2);
+            } else {
+              float x0, x1;
+              upk2(x2, x0, x1);
+              e2 = pk2(ex2(x0), ex2(x1));
+            }
+            acc2 = fadd2(acc2, e2);
+            float p0, p1;
+            upk2(e2, p0, p1);
             pk[i] = ptx::pack_bf16x2(p0, p1);
           }
           ptx::tmem_st16(tS + 16 * c, pk);
         }
+        float a0, a1;
+        upk2(acc2, a0, a1);
+        l_sum += a0 + a1;
       }
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
