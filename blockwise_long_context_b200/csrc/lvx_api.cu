@@ -154,15 +154,15 @@ lvx_status lvx_attn_bwd(const void* q, const void* k, const void* v, const void*
   const Problem p = make_problem(B, H, H_kv, S_Q, S_KV, d, 1, causal, scale);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const size_t row_bytes = align256((size_t)B * H * S_Q * sizeof(float));
-  float* D = reinterpret_cast<float*>(workspace);
-  float* lse2 = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) + row_bytes);
+  float* ND = reinterpret_cast<float*>(workspace);
+  float* nlse2 = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) + row_bytes);
   float* dq_acc = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) + 2 * row_bytes);
-  cudaError_t e = launch_bwd_pre(out, dout, lse, D, lse2, dq_acc, B, H, S_Q, d, dt, s);
+  cudaError_t e = launch_bwd_pre(out, dout, lse, ND, nlse2, dq_acc, B, H, S_Q, d, dt, s);
   if (e != cudaSuccess) return LVX_ERR_CUDA;
   if (dt == LVX_BF16 && tc_bwd_supported(p))
-    e = launch_bwd_tc(p, q, k, v, dout, lse2, D, dq_acc, dk, dv, s);
+    e = launch_bwd_tc(p, q, k, v, dout, nlse2, ND, dq_acc, dk, dv, s);
   else
-    e = launch_bwd_simt(p, dt, q, k, v, dout, lse, D, dq_acc, dk, dv, s);
+    e = launch_bwd_simt(p, dt, q, k, v, dout, lse, ND, dq_acc, dk, dv, s);
   if (e != cudaSuccess) return LVX_ERR_CUDA;
   return from_cuda(launch_dq_finalize(dq_acc, dq, (size_t)B * S_Q * H * d, p.scale, dt, s));
 }

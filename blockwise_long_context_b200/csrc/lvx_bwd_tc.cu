@@ -26,15 +26,17 @@
 namespace lvx {
 namespace {
 
+using namespace ptx;
+
 constexpr int BKEY = 128;
 constexpr int BROW = 128;
 constexpr int kThreads = 512;
 // Register split (launched at 128 per thread): warpgroup 0 (producer, MMA
-// issuer, allocator) 56, the two elementwise warpgroups 168, the dQ drain
-// warpgroup 120:  128 x 56 + 256 x 168 + 128 x 120 = 65536 = 512 x 128.
-constexpr uint32_t kRegsControl = 56;
+// issuer, allocator) 48, the two elementwise warpgroups 168, the dQ drain
+// warpgroup 128:  128 x 48 + 256 x 168 + 128 x 128 = 65536 = 512 x 128.
+constexpr uint32_t kRegsControl = 48;
 constexpr uint32_t kRegsElementwise = 168;
-constexpr uint32_t kRegsDrain = 120;
+constexpr uint32_t kRegsDrain = 128;
 static_assert(128 * kRegsControl + 256 * kRegsElementwise + 128 * kRegsDrain <=
                   65536 / kThreads * kThreads,
               "register split exceeds the launch allocation");
@@ -69,12 +71,6 @@ struct BwdArgs {
   int n_kt;   // key tiles per (batch, kv head)
   int n_qt;   // query tiles per head
 };
-
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
 
 // Adds a shared-memory tile into global memory through a tensor map (TMA
 // reduce-add in L2, asynchronous; the tile may be reused after bulk_wait_read).
@@ -115,11 +111,11 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
   uint64_t* dp_full = bars + 6;
   uint64_t* p_ready = bars + 7;
   uint64_t* ds_ready = bars + 8;
-  uint64_t* dv_done = bars + 9;
+  // bars[9] unused
   uint64_t* dq_full = bars + 10;
   uint64_t* dq_free = bars + 11;
   uint64_t* mma_drain = bars + 12;
-  uint64_t* stage_free = bars + 13;   // dQ staging (in the dS buffer) read back by the TMA
+  uint64_t* stage_free = bars + 13;   // dQ staging (in the dS buffer) read by the TMA
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -148,7 +144,6 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
     ptx::mbar_init(dp_full, 1);
     ptx::mbar_init(p_ready, 256);
     ptx::mbar_init(ds_ready, 256);
-    ptx::mbar_init(dv_done, 1);
     ptx::mbar_init(dq_full, 1);
     ptx::mbar_init(dq_free, 128);
     ptx::mbar_init(mma_drain, 1);
@@ -209,58 +204,80 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
         const uint32_t q_base = ptx::smem_u32(smem + L::OFF_Q);
         const uint32_t do_base = ptx::smem_u32(smem + L::OFF_DO);
         const uint32_t ds_base = ptx::smem_u32(smem + L::OFF_DS);
-        bool ok = ptx::mbar_wait(kv_full, 0, a.err, kErrTimeoutMma, abort_flag);
-        for (int i = 0; i < I && ok; ++i) {
-          const int s = i & 1;
-          ok = ptx::mbar_wait(&q_full[s], (i >> 1) & 1, a.err, kErrTimeoutMma, abort_flag);
-          if (ok && i > 0) ok = ptx::mbar_wait(dv_done, (i - 1) & 1, a.err, kErrTimeoutMma, abort_flag);
-          if (!ok) break;
-          ptx::tc_fence_after();
-          const uint32_t qs = q_base + s * L::TILE, dos = do_base + s * L::TILE;
-  #pragma unroll
+        // Issue order: S_0, dP_0, dV_0, then per tile i
+        //   S_{i+1}, dK_i, dQ_i, dP_{i+1}, dV_{i+1}.
+        // S_{i+1} goes right after dV_i, which reads P_i from the same TMEM
+        // columns: tcgen05.mma ops of one thread execute in issue order, so the
+        // read completes first, and the elementwise warps can start on tile
+        // i+1 while the tensor core works on dK_i and dQ_i.  dP_{i+1} reuses the
+        // columns of dQ_i and waits until the drain warps have read them.
+        auto issue_s = [&](int i) {
+          const uint32_t qs = q_base + (i & 1) * L::TILE;
+#pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {   // S^T = K Q^T
             const uint32_t off = (kk >> 2) * CHUNK + (kk & 3) * 32;
             ptx::mma_ss(tS, ptx::smem_desc_sw128(k_base + off, 16, 1024),
                         ptx::smem_desc_sw128(qs + off, 16, 1024), L::IDESC_SS_KK, kk > 0);
           }
           ptx::mma_commit(s_full);
-          if (i > 0) {
-            ok = ptx::mbar_wait(dq_free, (i - 1) & 1, a.err, kErrTimeoutMma, abort_flag);
-            if (!ok) break;
-            ptx::tc_fence_after();
-          }
-  #pragma unroll
+        };
+        auto issue_dp_dv = [&](int i) -> bool {
+          const uint32_t dos = do_base + (i & 1) * L::TILE;
+#pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {   // dP^T = V dO^T
             const uint32_t off = (kk >> 2) * CHUNK + (kk & 3) * 32;
             ptx::mma_ss(tdP, ptx::smem_desc_sw128(v_base + off, 16, 1024),
                         ptx::smem_desc_sw128(dos + off, 16, 1024), L::IDESC_SS_KK, kk > 0);
           }
           ptx::mma_commit(dp_full);
-          ok = ptx::mbar_wait(p_ready, i & 1, a.err, kErrTimeoutMma, abort_flag);
-          if (!ok) break;
+          if (!ptx::mbar_wait(p_ready, i & 1, a.err, kErrTimeoutMma, abort_flag)) return false;
           ptx::tc_fence_after();
-  #pragma unroll
+#pragma unroll
           for (int kk = 0; kk < BROW / 16; ++kk)   // dV += P^T dO (P^T halves at columns 0 and 64)
             ptx::mma_ts(tdV, tS + (kk >> 2) * 64 + (kk & 3) * 8,
                         ptx::smem_desc_sw128(dos + kk * 2048, CHUNK, 1024),
                         L::IDESC_DV, (i > 0 || kk > 0) ? 1u : 0u);
-          ptx::mma_commit(dv_done);
+          return true;
+        };
+        bool ok = I > 0 && ptx::mbar_wait(kv_full, 0, a.err, kErrTimeoutMma, abort_flag);
+        if (ok) ok = ptx::mbar_wait(&q_full[0], 0, a.err, kErrTimeoutMma, abort_flag);
+        if (ok) {
+          ptx::tc_fence_after();
+          issue_s(0);
+          ok = issue_dp_dv(0);
+        }
+        for (int i = 0; i < I && ok; ++i) {
+          const int s = i & 1;
+          if (i + 1 < I) {
+            ok = ptx::mbar_wait(&q_full[(i + 1) & 1], ((i + 1) >> 1) & 1, a.err, kErrTimeoutMma,
+                                abort_flag);
+            if (!ok) break;
+            ptx::tc_fence_after();
+            issue_s(i + 1);
+          }
           ok = ptx::mbar_wait(ds_ready, i & 1, a.err, kErrTimeoutMma, abort_flag);
           if (!ok) break;
           ptx::tc_fence_after();
-  #pragma unroll
+          const uint32_t qs = q_base + s * L::TILE;
+#pragma unroll
           for (int kk = 0; kk < BROW / 16; ++kk) {   // dK += dS^T Q
             const uint32_t off = (kk >> 2) * CHUNK + (kk & 3) * 32;
             ptx::mma_ss(tdK, ptx::smem_desc_sw128(ds_base + off, 16, 1024),
                         ptx::smem_desc_sw128(qs + kk * 2048, CHUNK, 1024), L::IDESC_DK,
                         (i > 0 || kk > 0) ? 1u : 0u);
           }
-  #pragma unroll
+#pragma unroll
           for (int kk = 0; kk < BKEY / 16; ++kk)   // dQ_t = dS K
             ptx::mma_ss(tdP, ptx::smem_desc_sw128(ds_base + kk * 2048, CHUNK, 1024),
                         ptx::smem_desc_sw128(k_base + kk * 2048, CHUNK, 1024), L::IDESC_DQ, kk > 0);
           ptx::mma_commit(dq_full);
           ptx::mma_commit(&q_empty[s]);
+          if (i + 1 < I) {
+            ok = ptx::mbar_wait(dq_free, i & 1, a.err, kErrTimeoutMma, abort_flag);
+            if (!ok) break;
+            ptx::tc_fence_after();
+            ok = issue_dp_dv(i + 1);
+          }
         }
         ptx::mma_commit(mma_drain);
       }
@@ -281,9 +298,9 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
       const int h = g * grp + i / per_head;
       const int m = m_start + i % per_head;
       const int r0 = BROW * m + 64 * hf;       // first query row handled by this thread
-      // the LSE stage holds LSE * log2(e) (scaled by the preprocess kernel)
-      const float* lse_s = reinterpret_cast<const float*>(smem + L::OFF_LSE + s * 512) + 64 * hf;
-      const float* dd_s = reinterpret_cast<const float*>(smem + L::OFF_DD + s * 512) + 64 * hf;
+      // the stages hold -LSE*log2(e) and -rowsum(dO o O) (written by the preprocess kernel)
+      const float* nlse_s = reinterpret_cast<const float*>(smem + L::OFF_LSE + s * 512) + 64 * hf;
+      const float* nd_s = reinterpret_cast<const float*>(smem + L::OFF_DD + s * 512) + 64 * hf;
       // this stage's LSE and D rows (TMA) are read directly below; the stage is
       // only refilled after the MMAs of this tile, which wait for this thread
       ok = ptx::mbar_wait(&q_full[s], (i >> 1) & 1, a.err, kErrTimeoutSoftmax, abort_flag);
@@ -291,7 +308,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       ptx::tc_fence_after();
-      float P[64];
+      uint64_t P2[32];   // P^T of this thread's 64 query rows as packed fp32 pairs
       {
         uint32_t sr[64];
         ptx::tmem_ld32(tS + lane_off + 64 * hf, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
@@ -303,20 +320,47 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
         if (need_mask) {
           const bool key_ok = key < p.S_KV;
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            const int r = r0 + c;
-            const bool vis = key_ok && r < p.S_Q && (!p.causal || key <= r);
-            P[c] = vis ? ex2(fmaf(__uint_as_float(sr[c]), sl2, -lse_s[c])) : 0.f;
+          for (int c = 0; c < 32; ++c) {
+            float e[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int r = r0 + 2 * c + u;
+              const bool vis = key_ok && r < p.S_Q && (!p.causal || key <= r);
+              e[u] = vis ? ex2(fmaf(__uint_as_float(sr[2 * c + u]), sl2, nlse_s[2 * c + u])) : 0.f;
+            }
+            P2[c] = pk2(e[0], e[1]);
           }
         } else {
+          // x = s * scale*log2(e) - LSE*log2(e) on FFMA2; one pair in kPolyEvery of the
+          // exponentials on the FMA pipe, the rest on the SFU
+          const uint64_t sl2x2 = pk2(sl2, sl2);
 #pragma unroll
-          for (int c = 0; c < 64; ++c) P[c] = ex2(fmaf(__uint_as_float(sr[c]), sl2, -lse_s[c]));
+          for (int c4 = 0; c4 < 16; ++c4) {
+            const float4 l4 = *reinterpret_cast<const float4*>(nlse_s + 4 * c4);
+            const uint64_t xa = ffma2(pk2(__uint_as_float(sr[4 * c4]), __uint_as_float(sr[4 * c4 + 1])),
+                                      sl2x2, pk2(l4.x, l4.y));
+            const uint64_t xb = ffma2(pk2(__uint_as_float(sr[4 * c4 + 2]), __uint_as_float(sr[4 * c4 + 3])),
+                                      sl2x2, pk2(l4.z, l4.w));
+            float a0, a1, b0, b1;
+            upk2(xa, a0, a1);
+            P2[2 * c4] = pk2(ex2(a0), ex2(a1));
+            if ((2 * c4 + 1) % kPolyEvery == kPolyEvery - 1) {
+              P2[2 * c4 + 1] = exp2_poly2(xb);
+            } else {
+              upk2(xb, b0, b1);
+              P2[2 * c4 + 1] = pk2(ex2(b0), ex2(b1));
+            }
+          }
         }
       }
       {
         uint32_t pk[32];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) pk[c] = ptx::pack_bf16x2(P[2 * c], P[2 * c + 1]);
+        for (int c = 0; c < 32; ++c) {
+          float lo, hi;
+          upk2(P2[c], lo, hi);
+          pk[c] = ptx::pack_bf16x2(lo, hi);
+        }
         // P^T of rows [64hf, 64hf+64) goes to columns [64hf, 64hf+32): only over
         // S^T columns this thread has already read
         ptx::tmem_st32(tS + lane_off + 64 * hf, pk);
@@ -325,15 +369,15 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
       ptx::tc_fence_before();
       ptx::mbar_arrive(p_ready);
       ok = ptx::mbar_wait(dp_full, i & 1, a.err, kErrTimeoutSoftmax, abort_flag);
-      // the dS buffer doubles as the drain's dQ staging: wait until the drain
-      // warps' TMA reductions of the previous tile have read it
+      // the dS buffer doubles as the drain's dQ staging: wait until the TMA has
+      // read the previous tile's pieces
       if (ok && i > 0)
         ok = ptx::mbar_wait(stage_free, (i - 1) & 1, a.err, kErrTimeoutSoftmax, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       ptx::tc_fence_after();
       // dS^T row of key j, query rows r0 .. r0+63 (one 128-byte swizzled row),
-      // in two 32-column halves to bound register use
+      // dS = P o (dP - D) on FADD2/FMUL2, in two 32-column halves to bound registers
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t dr[32];
@@ -342,16 +386,20 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
 #pragma unroll
         for (int q8 = 0; q8 < 4; ++q8) {
           const int c8 = 4 * half + q8;
-          float e[8];
+          const float4 na = *reinterpret_cast<const float4*>(nd_s + 8 * c8);
+          const float4 nb = *reinterpret_cast<const float4*>(nd_s + 8 * c8 + 4);
+          const float nv[8] = {na.x, na.y, na.z, na.w, nb.x, nb.y, nb.z, nb.w};
+          uint32_t w[4];
 #pragma unroll
-          for (int t = 0; t < 8; ++t)
-            e[t] = P[8 * c8 + t] * (__uint_as_float(dr[8 * q8 + t]) - dd_s[8 * c8 + t]);
-          uint4 u;
-          u.x = ptx::pack_bf16x2(e[0], e[1]);
-          u.y = ptx::pack_bf16x2(e[2], e[3]);
-          u.z = ptx::pack_bf16x2(e[4], e[5]);
-          u.w = ptx::pack_bf16x2(e[6], e[7]);
-          *reinterpret_cast<uint4*>(ds_smem + ((c8 ^ (j & 7)) << 4)) = u;
+          for (int t = 0; t < 4; ++t) {
+            const uint64_t d2 = fadd2(pk2(__uint_as_float(dr[8 * q8 + 2 * t]),
+                                          __uint_as_float(dr[8 * q8 + 2 * t + 1])),
+                                      pk2(nv[2 * t], nv[2 * t + 1]));
+            float e0, e1;
+            upk2(fmul2(P2[4 * c8 + t], d2), e0, e1);
+            w[t] = ptx::pack_bf16x2(e0, e1);
+          }
+          *reinterpret_cast<uint4*>(ds_smem + ((c8 ^ (j & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
       ptx::fence_proxy_async_smem();
@@ -473,6 +521,14 @@ cudaError_t launch(const Problem& p, const void* q, const void* k, const void* v
                    void* dv, cudaStream_t s) {
   using L = BwdLayout<D>;
   CUtensorMap mq, mk, mv, mdo, mlse, mdd, mdq;
+  {
+    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)p.H, (uint64_t)p.S_Q, (uint64_t)p.B};
+    const uint64_t str[3] = {(uint64_t)D * 4, (uint64_t)p.H * D * 4, (uint64_t)p.S_Q * p.H * D * 4};
+    const uint32_t box4[4] = {32, 1, 32, 1};
+    if (!encode_tensor_map(&mdq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dq_acc, dims, str, box4,
+                           CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  }
   const uint32_t box[4] = {64, 1, 128, 1};
   {
     const uint64_t dims[4] = {(uint64_t)D, (uint64_t)p.H, (uint64_t)p.S_Q, (uint64_t)p.B};
@@ -504,14 +560,6 @@ cudaError_t launch(const Problem& p, const void* q, const void* k, const void* v
                            CU_TENSOR_MAP_SWIZZLE_NONE))
       return cudaErrorInvalidValue;
   }
-  {
-    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)p.H, (uint64_t)p.S_Q, (uint64_t)p.B};
-    const uint64_t str[3] = {(uint64_t)D * 4, (uint64_t)p.H * D * 4, (uint64_t)p.S_Q * p.H * D * 4};
-    const uint32_t box4[4] = {32, 1, 32, 1};
-    if (!encode_tensor_map(&mdq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dq_acc, dims, str, box4,
-                           CU_TENSOR_MAP_SWIZZLE_128B))
-      return cudaErrorInvalidValue;
-  }
   BwdArgs a;
   a.p = p;
   a.dq_acc = dq_acc;
@@ -536,10 +584,10 @@ cudaError_t launch(const Problem& p, const void* q, const void* k, const void* v
 bool tc_bwd_supported(const Problem& p) { return (p.d == 64 || p.d == 128) && p.S_Q % 4 == 0; }
 
 cudaError_t launch_bwd_tc(const Problem& p, const void* q, const void* k, const void* v,
-                          const void* dout, const float* lse, const float* D, float* dq_acc,
+                          const void* dout, const float* nlse2, const float* nd, float* dq_acc,
                           void* dk, void* dv, cudaStream_t s) {
-  if (p.d == 128) return launch<128>(p, q, k, v, dout, lse, D, dq_acc, dk, dv, s);
-  if (p.d == 64) return launch<64>(p, q, k, v, dout, lse, D, dq_acc, dk, dv, s);
+  if (p.d == 128) return launch<128>(p, q, k, v, dout, nlse2, nd, dq_acc, dk, dv, s);
+  if (p.d == 64) return launch<64>(p, q, k, v, dout, nlse2, nd, dq_acc, dk, dv, s);
   return cudaErrorInvalidValue;
 }
 

@@ -61,11 +61,11 @@ cudaError_t launch_fwd_simt(const Problem& p, lvx_dtype dt, const void* q, const
 cudaError_t launch_merge(const float* o_parts, const float* l_parts, void* out, float* lse,
                          int n, int B, int H, int S_Q, int d, int causal, int block_len,
                          lvx_dtype dt, cudaStream_t s);
-cudaError_t launch_bwd_pre(const void* out, const void* dout, const float* lse, float* D,
-                           float* lse2, float* dq_acc, int B, int H, int S_Q, int d, lvx_dtype dt,
+cudaError_t launch_bwd_pre(const void* out, const void* dout, const float* lse, float* ND,
+                           float* nlse2, float* dq_acc, int B, int H, int S_Q, int d, lvx_dtype dt,
                            cudaStream_t s);
 cudaError_t launch_bwd_simt(const Problem& p, lvx_dtype dt, const void* q, const void* k,
-                            const void* v, const void* dout, const float* lse, const float* D,
+                            const void* v, const void* dout, const float* lse, const float* ND,
                             float* dq_acc, void* dk, void* dv, cudaStream_t s);
 cudaError_t launch_dq_finalize(const float* dq_acc, void* dq, size_t count, float scale,
                                lvx_dtype dt, cudaStream_t s);

@@ -103,14 +103,15 @@ merge_kernel(const float* __restrict__ o_parts, const float* __restrict__ l_part
   }
 }
 
-// D[b,h,r] = sum_c dO[b,r,h,c] * O[b,r,h,c] and LSE2[b,h,r] = LSE[b,h,r] * log2(e)
-// (the tensor-core backward exponentiates with exp2); also clears dq_acc.  Rows are
+// ND[b,h,r] = -sum_c dO[b,r,h,c] * O[b,r,h,c] (minus D of the gradient) and
+// NLSE2[b,h,r] = -LSE[b,h,r] * log2(e) (the tensor-core backward exponentiates with
+// exp2 and adds both with packed FMAs); also clears dq_acc.  Rows are
 // taken in memory order [B, S_Q, H]; a row's d/8 threads form an aligned
 // power-of-two lane group of one warp and reduce with xor shuffles.
 template <typename T>
 __global__ void __launch_bounds__(256)
 bwd_pre_kernel(const T* __restrict__ out, const T* __restrict__ dout, const float* __restrict__ lse,
-               float* __restrict__ D, float* __restrict__ lse2, float* __restrict__ dq_acc, int B,
+               float* __restrict__ ND, float* __restrict__ nlse2, float* __restrict__ dq_acc, int B,
                int H, int S_Q, int d) {
   const int tpr = d / 8;
   int G = 1;
@@ -140,8 +141,8 @@ bwd_pre_kernel(const T* __restrict__ out, const T* __restrict__ dout, const floa
       const size_t bs = row / H;
       const int r = (int)(bs % S_Q), b = (int)(bs / S_Q);
       const size_t o = ((size_t)b * H + h) * S_Q + r;
-      D[o] = part;
-      lse2[o] = lse[o] * kLog2e;
+      ND[o] = -part;
+      nlse2[o] = -lse[o] * kLog2e;
     }
   }
 }
@@ -184,17 +185,17 @@ cudaError_t launch_merge(const float* o_parts, const float* l_parts, void* out, 
   return cudaGetLastError();
 }
 
-cudaError_t launch_bwd_pre(const void* out, const void* dout, const float* lse, float* D,
-                           float* lse2, float* dq_acc, int B, int H, int S_Q, int d, lvx_dtype dt,
+cudaError_t launch_bwd_pre(const void* out, const void* dout, const float* lse, float* ND,
+                           float* nlse2, float* dq_acc, int B, int H, int S_Q, int d, lvx_dtype dt,
                            cudaStream_t s) {
   const size_t work = (size_t)B * H * S_Q * (d / 8);
   const int grid = grid_for(work, 256);
   if (dt == LVX_FP32)
-    bwd_pre_kernel<float><<<grid, 256, 0, s>>>((const float*)out, (const float*)dout, lse, D, lse2,
+    bwd_pre_kernel<float><<<grid, 256, 0, s>>>((const float*)out, (const float*)dout, lse, ND, nlse2,
                                                dq_acc, B, H, S_Q, d);
   else
     bwd_pre_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>((const __nv_bfloat16*)out,
-                                                       (const __nv_bfloat16*)dout, lse, D, lse2,
+                                                       (const __nv_bfloat16*)dout, lse, ND, nlse2,
                                                        dq_acc, B, H, S_Q, d);
   return cudaGetLastError();
 }

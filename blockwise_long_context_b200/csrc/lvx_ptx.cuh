@@ -261,6 +261,80 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_ma
          | ((uint32_t)(M >> 4) << 24);               // M / 16
 }
 
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Packed fp32 pairs (Blackwell FFMA2 / FADD2) and the three-input maximum.
+__device__ __forceinline__ uint64_t pk2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void upk2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x on the FMA pipe: x = n + f with n = round(x), |f| <= 1/2; 2^f from a
+// cubic fitted by fit_exp2.py (max relative error 7.5e-5, far below the
+// bf16 rounding P receives); n is added to the exponent field.  Adding
+// 1.5 * 2^23 leaves round(x) in the low mantissa bits of t.  x is clamped at
+// -127 so the exponent cannot wrap; callers use it only on unmasked tiles,
+// where the argument is finite.
+constexpr int kPolyEvery = 4;   // one pair of exponentials in kPolyEvery on the FMA pipe
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -127.f);
+  const float t = x + 12582912.f;
+  const float f = x - (t - 12582912.f);
+  const float p = fmaf(fmaf(fmaf(5.517164990e-02f, f, 2.426111400e-01f), f, 6.932609677e-01f), f,
+                       9.999280572e-01f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// The same for a packed pair, with the fp32 arithmetic on FFMA2 / FADD2.
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
+  float x0, x1;
+  upk2(x2, x0, x1);
+  x2 = pk2(fmaxf(x0, -127.f), fmaxf(x1, -127.f));
+  const uint64_t magic = pk2(12582912.f, 12582912.f);
+  const uint64_t nmagic = pk2(-12582912.f, -12582912.f);
+  const uint64_t t = fadd2(x2, magic);
+  const uint64_t r = fadd2(t, nmagic);
+  float r0, r1;
+  upk2(r, r0, r1);
+  const uint64_t f = fadd2(x2, pk2(-r0, -r1));
+  uint64_t p = ffma2(pk2(5.517164990e-02f, 5.517164990e-02f), f, pk2(2.426111400e-01f, 2.426111400e-01f));
+  p = ffma2(p, f, pk2(6.932609677e-01f, 6.932609677e-01f));
+  p = ffma2(p, f, pk2(9.999280572e-01f, 9.999280572e-01f));
+  float p0, p1, t0, t1;
+  upk2(p, p0, p1);
+  upk2(t, t0, t1);
+  return pk2(__int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23)),
+             __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23)));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));

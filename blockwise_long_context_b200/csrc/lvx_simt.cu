@@ -143,7 +143,7 @@ template <typename T>
 __global__ void __launch_bounds__(128)
 bwd_simt_kernel(Problem p, const T* __restrict__ q, const T* __restrict__ k,
                 const T* __restrict__ v, const T* __restrict__ dout,
-                const float* __restrict__ lse, const float* __restrict__ D,
+                const float* __restrict__ lse, const float* __restrict__ ND,
                 float* __restrict__ dq_acc, T* __restrict__ dk, T* __restrict__ dv) {
   __shared__ float ks[kBwdKeys][kMaxD];
   __shared__ float vs[kBwdKeys][kMaxD];
@@ -189,7 +189,7 @@ bwd_simt_kernel(Problem p, const T* __restrict__ q, const T* __restrict__ k,
         dqv[t] = 0.f;
       }
       const float L2 = lse[((size_t)b * p.H + h) * p.S_Q + r] * lse_scale;
-      const float Dr = D[((size_t)b * p.H + h) * p.S_Q + r];
+      const float NDr = ND[((size_t)b * p.H + h) * p.S_Q + r];   // minus rowsum(dO o O)
 #pragma unroll
       for (int jj = 0; jj < kBwdKeysPerWarp; ++jj) {
         const int j = k0 + jw + jj;
@@ -206,7 +206,7 @@ bwd_simt_kernel(Problem p, const T* __restrict__ q, const T* __restrict__ k,
         pdot = warp_sum(pdot);
         const bool visible = j < p.S_KV && (!p.causal || j <= r);
         const float P = visible ? exp2f(sdot * p.scale_log2 - L2) : 0.f;
-        const float dS = P * (pdot - Dr);
+        const float dS = P * (pdot + NDr);
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
           const int c = lane + 32 * t;
@@ -299,17 +299,17 @@ cudaError_t launch_fwd_simt(const Problem& p, lvx_dtype dt, const void* q, const
 }
 
 cudaError_t launch_bwd_simt(const Problem& p, lvx_dtype dt, const void* q, const void* k,
-                            const void* v, const void* dout, const float* lse, const float* D,
+                            const void* v, const void* dout, const float* lse, const float* ND,
                             float* dq_acc, void* dk, void* dv, cudaStream_t s) {
   dim3 grid((p.S_KV + kBwdKeys - 1) / kBwdKeys, p.B * p.H_kv);
   if (dt == LVX_FP32)
     bwd_simt_kernel<float><<<grid, 32 * kBwdWarps, 0, s>>>(p, (const float*)q, (const float*)k,
-                                                (const float*)v, (const float*)dout, lse, D,
+                                                (const float*)v, (const float*)dout, lse, ND,
                                                 dq_acc, (float*)dk, (float*)dv);
   else
     bwd_simt_kernel<__nv_bfloat16><<<grid, 32 * kBwdWarps, 0, s>>>(
         p, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
-        (const __nv_bfloat16*)dout, lse, D, dq_acc, (__nv_bfloat16*)dk, (__nv_bfloat16*)dv);
+        (const __nv_bfloat16*)dout, lse, ND, dq_acc, (__nv_bfloat16*)dk, (__nv_bfloat16*)dv);
   return cudaGetLastError();
 }
 

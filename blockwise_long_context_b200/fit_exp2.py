@@ -11,7 +11,7 @@ iteratively reweighted least squares on Chebyshev nodes.
 
 prints the fp32 coefficients (c0, c1, c2, c3) and the maximum relative
 error of the fp32 Horner evaluation; the values are embedded in
-csrc/lvx_fwd_tc.cu and a CPU test re-runs this fit to check them.
+csrc/lvx_ptx.cuh and a CPU test re-runs this fit to check them.
 """
 
 import numpy as np

@@ -145,8 +145,8 @@ lvx_status lvx_merge_partials(const float* O_parts, const float* L_parts, void* 
 
 /*
  * Workspace bytes for lvx_attn_bwd.  Layout (256-byte aligned parts):
- *   D      [B, H, S_Q]      float32  rowsum(dO o O)
- *   LSE2   [B, H, S_Q]      float32  lse * log2(e)
+ *   ND     [B, H, S_Q]      float32  -rowsum(dO o O)
+ *   NLSE2  [B, H, S_Q]      float32  -lse * log2(e)
  *   dQ_acc [B, S_Q, H, d]   float32  unscaled dQ accumulator
  */
 size_t lvx_attn_bwd_workspace(int B, int H, int H_kv, int S_Q, int S_KV, int d,
