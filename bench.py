@@ -39,7 +39,11 @@ WORKLOAD = "C2"
 
 # ncu DRAM traffic of the dominant kernel per launch, with the hash of the
 # source file it was taken from (reported only while the source is unchanged).
-TRAFFIC = {}
+TRAFFIC = {
+    # bwd_tc_kernel, full C2 launch: 336.32 MB read + 251.76 MB written (profiles/dram_traffic_c2_full.md)
+    "bwd": {"bytes": 588.08e6, "source": "blockwise_long_context_b200/csrc/lvx_bwd_tc.cu",
+            "sha": "229e1c412465084d"},
+}
 
 
 def _peaks():
@@ -176,6 +180,24 @@ def _config(w, n):
                              "2*2*B*S_KV*d_embed*H_kv*d"}
 
 
+# ---------------------------------------------------------------- multi-rank helpers
+
+def max_over_ranks(x: float, device) -> float:
+    """Max of a per-rank device time over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flops_per_rank_step: float, steps: int, world: int, ms: float) -> float:
+    """Weak scaling: every rank does the same work; the slowest rank sets the time."""
+    return world * flops_per_rank_step * steps / (ms * 1e-3) / 1e12
+
+
 # ---------------------------------------------------------------- GPU arm
 
 def _file_sha(rel):
@@ -253,13 +275,10 @@ def run_gpu(a):
     t_bwd = statistics.mean(ev[2].elapsed_time(ev[3]) for ev in stage_ev)
     lvx.lvx_last_device_error()
 
-    if world > 1:
-        t = torch.tensor([ms_total], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(ms_total, dev)
     ms_step = ms_total / a.steps
     step_flops = w.fwd_flops() + w.bwd_flops() + w.kv_flops()
-    value = world * step_flops * a.steps / (ms_total * 1e-3) / 1e12
+    value = whole_job_tflops(step_flops, a.steps, world, ms_total)
 
     # merge kernel alone (HBM-bound), after an L2 flush, through the merge entry point
     flush = torch.empty(256 * 2**20, dtype=torch.uint8, device=dev)
@@ -299,11 +318,8 @@ def run_gpu(a):
     x1.record(stream)
     torch.cuda.synchronize()
     ms_e2e = x0.elapsed_time(x1)
-    if world > 1:
-        t = torch.tensor([ms_e2e], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_e2e = float(t.item())
-    e2e_value = world * step_flops * n_e2e / (ms_e2e * 1e-3) / 1e12
+    ms_e2e = max_over_ranks(ms_e2e, dev)
+    e2e_value = whole_job_tflops(step_flops, n_e2e, world, ms_e2e)
 
     # roofline of the dominant kernel group (timed inside the long step loop: sustained peak)
     stages = {"bwd": (t_bwd, w.bwd_flops(), "lvx_attn_bwd (preprocess + main + dQ finalize)"),

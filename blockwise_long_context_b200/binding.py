@@ -44,6 +44,7 @@ _SIGS = {
     "lvx_attn_bwd": ([_vp] * 9 + [_c_int] * 7 + [_c_int, _c_float, _vp, _c_size, _vp], _c_int),
     "lvx_kv_recompute": ([_vp] * 5 + [_c_int] * 5 + [_c_int, _vp], _c_int),
     "lvx_last_device_error": ([_vp], _c_int),
+    "lvx_selftest_wait_timeout": ([_vp], _c_int),
 }
 
 
@@ -151,6 +152,10 @@ def lvx_kv_recompute(y, w_k, w_v, k, v, H_kv: int, d: int, stream=None) -> None:
 
 def lvx_last_device_error(stream=None) -> None:
     _check(lib().lvx_last_device_error(_stream(stream)), "lvx_last_device_error")
+
+
+def lvx_selftest_wait_timeout(stream=None) -> None:
+    _check(lib().lvx_selftest_wait_timeout(_stream(stream)), "lvx_selftest_wait_timeout")
 
 
 # ------------------------------------------------------------------ conveniences

@@ -31,6 +31,7 @@ enum : unsigned int {
   kErrTimeoutSoftmax = 3,
   kErrTimeoutEpilogue = 4,
   kErrSmemAlign = 5,
+  kErrSelftestTimeout = 6,
 };
 
 __device__ __forceinline__ void record_error(unsigned int* word, unsigned int code) {

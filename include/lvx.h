@@ -196,6 +196,16 @@ lvx_status lvx_kv_recompute(const void* y, const void* w_k, const void* w_v, voi
  */
 lvx_status lvx_last_device_error(lvx_stream stream);
 
+/*
+ * Diagnostic: launches one small kernel that waits on a barrier nothing ever
+ * completes.  Its bounded wait gives up after about 2 s, records a timeout in
+ * the device error word and returns, exactly as the library's tensor-core
+ * kernels do when an internal wait expires; the next lvx_last_device_error
+ * then returns LVX_ERR_DEVICE_TIMEOUT and the context stays usable.  (Not part
+ * of the attention method; used to test the failure path without a fault.)
+ */
+lvx_status lvx_selftest_wait_timeout(lvx_stream stream);
+
 #ifdef __cplusplus
 }
 #endif
