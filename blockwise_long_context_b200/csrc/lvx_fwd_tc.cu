@@ -11,7 +11,7 @@
 // exponentials stay below 256, so the deferred rescaling is exact).
 //
 // Roles (12 warps):
-//   warp 0      TMA producer: Q tiles once, K and V tiles through 2-stage rings
+//   warp 0      TMA producer: Q tiles once, K (3-stage) and V (2-stage) rings
 //   warp 1      MMA issuer:   S_t = Q_t K^T (SS form) and O_t += P_t V (TS form,
 //                             P read from TMEM)
 //   warp 2      TMEM allocator (512 columns)
@@ -32,7 +32,8 @@ using namespace ptx;
 constexpr int BQ = 128;           // query rows per tile (MMA M)
 constexpr int BKV = 128;          // keys per tile
 constexpr int NQT = 2;            // query tiles per CTA
-constexpr int KV_STAGES = 2;
+constexpr int K_STAGES = 3;   // K is needed a full softmax earlier than V: prefetch it deeper
+constexpr int V_STAGES = 2;
 constexpr int kThreads = 384;
 // Register split: launched at 168 per thread (384 x 168 = 64512); warpgroup 0
 // (producer, MMA issuer, allocator) gives up 64, the two softmax warpgroups
@@ -50,8 +51,8 @@ struct FwdLayout {
   static constexpr uint32_t TILE = 128 * D * 2;   // Q, K or V tile
   static constexpr uint32_t OFF_Q = 0;
   static constexpr uint32_t OFF_K = OFF_Q + NQT * TILE;
-  static constexpr uint32_t OFF_V = OFF_K + KV_STAGES * TILE;
-  static constexpr uint32_t OFF_BAR = OFF_V + KV_STAGES * TILE;
+  static constexpr uint32_t OFF_V = OFF_K + K_STAGES * TILE;
+  static constexpr uint32_t OFF_BAR = OFF_V + V_STAGES * TILE;
   static constexpr uint32_t USED = OFF_BAR + 256 + 1024;
   // at least ~116 KiB so that one CTA (and its 512 TMEM columns) owns the SM
   static constexpr uint32_t BYTES = USED > 118784 ? USED : 118784;
@@ -79,15 +80,15 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;
-  uint64_t* k_empty = bars + 3;
-  uint64_t* v_full = bars + 5;
-  uint64_t* v_empty = bars + 7;
-  uint64_t* s_full = bars + 9;
-  uint64_t* p_full = bars + 11;
-  uint64_t* o_done = bars + 13;
-  uint64_t* mma_drain = bars + 15;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  uint64_t* k_full = bars + 1;     // [K_STAGES]
+  uint64_t* k_empty = bars + 4;    // [K_STAGES]
+  uint64_t* v_full = bars + 7;     // [V_STAGES]
+  uint64_t* v_empty = bars + 9;    // [V_STAGES]
+  uint64_t* s_full = bars + 11;
+  uint64_t* p_full = bars + 13;
+  uint64_t* o_done = bars + 15;
+  uint64_t* mma_drain = bars + 17;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const Problem& p = a.p;
@@ -113,9 +114,11 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     ptx::mbar_init(q_full, 1);
-    for (int s = 0; s < KV_STAGES; ++s) {
+    for (int s = 0; s < K_STAGES; ++s) {
       ptx::mbar_init(&k_full[s], 1);
       ptx::mbar_init(&k_empty[s], 1);
+    }
+    for (int s = 0; s < V_STAGES; ++s) {
       ptx::mbar_init(&v_full[s], 1);
       ptx::mbar_init(&v_empty[s], 1);
     }
@@ -150,30 +153,37 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
             ptx::tma_load_4d(smem + L::OFF_Q + t * L::TILE + c * CHUNK, &map_q, q_full, 64 * c, h,
                              m0 + BQ * t, b);
         int issued_k = 0, issued_v = 0;
-        for (int j = 0; j < T; ++j) {
-          const int s = j & 1;
-          const uint32_t ph = ((j >> 1) & 1) ^ 1;
-          const int key0 = kb0 + BKV * j;
-          if (!ptx::mbar_wait(&k_empty[s], ph, a.err, kErrTimeoutTma, abort_flag)) break;
+        auto load_k = [&](int j) -> bool {
+          const int s = j % K_STAGES;
+          if (!ptx::mbar_wait(&k_empty[s], ((j / K_STAGES) & 1) ^ 1, a.err, kErrTimeoutTma, abort_flag))
+            return false;
           ptx::mbar_arrive_expect_tx(&k_full[s], L::TILE);
           for (int c = 0; c < D / 64; ++c)
             ptx::tma_load_4d(smem + L::OFF_K + s * L::TILE + c * CHUNK, &map_k, &k_full[s], 64 * c,
-                             g, key0, b);
+                             g, kb0 + BKV * j, b);
           issued_k = j + 1;
-          if (!ptx::mbar_wait(&v_empty[s], ph, a.err, kErrTimeoutTma, abort_flag)) break;
+          return true;
+        };
+        // order K_0, then per j: K_{j+1}, V_j -- keys run ahead of values
+        bool ok = load_k(0);
+        for (int j = 0; j < T && ok; ++j) {
+          if (j + 1 < T && !load_k(j + 1)) break;
+          const int s = j % V_STAGES;
+          if (!ptx::mbar_wait(&v_empty[s], ((j / V_STAGES) & 1) ^ 1, a.err, kErrTimeoutTma, abort_flag))
+            break;
           ptx::mbar_arrive_expect_tx(&v_full[s], L::TILE);
           for (int c = 0; c < D / 64; ++c)
             ptx::tma_load_4d(smem + L::OFF_V + s * L::TILE + c * CHUNK, &map_v, &v_full[s], 64 * c,
-                             g, key0, b);
+                             g, kb0 + BKV * j, b);
           issued_v = j + 1;
         }
         if (*abort_flag) {
           // the copies already issued must land before shared memory is released
           ptx::mbar_wait(q_full, 0, a.err, kErrTimeoutTma, nullptr);
-          for (int j = issued_k > KV_STAGES ? issued_k - KV_STAGES : 0; j < issued_k; ++j)
-            ptx::mbar_wait(&k_full[j & 1], (j >> 1) & 1, a.err, kErrTimeoutTma, nullptr);
-          for (int j = issued_v > KV_STAGES ? issued_v - KV_STAGES : 0; j < issued_v; ++j)
-            ptx::mbar_wait(&v_full[j & 1], (j >> 1) & 1, a.err, kErrTimeoutTma, nullptr);
+          for (int j = issued_k > K_STAGES ? issued_k - K_STAGES : 0; j < issued_k; ++j)
+            ptx::mbar_wait(&k_full[j % K_STAGES], (j / K_STAGES) & 1, a.err, kErrTimeoutTma, nullptr);
+          for (int j = issued_v > V_STAGES ? issued_v - V_STAGES : 0; j < issued_v; ++j)
+            ptx::mbar_wait(&v_full[j % V_STAGES], (j / V_STAGES) & 1, a.err, kErrTimeoutTma, nullptr);
         }
       }
     } else if (warp == 1) {
@@ -191,7 +201,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
           const uint32_t k_base = ptx::smem_u32(smem + L::OFF_K);
           const uint32_t v_base = ptx::smem_u32(smem + L::OFF_V);
           auto issue_s = [&](int t, int j) {
-            const int s = j & 1;
+            const int s = j % K_STAGES;
   #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               const uint32_t off = (kk >> 2) * CHUNK + (kk & 3) * 32;
@@ -202,7 +212,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
             ptx::mma_commit(&s_full[t]);
           };
           auto issue_pv = [&](int t, int j) {
-            const int s = j & 1;
+            const int s = j % V_STAGES;
   #pragma unroll
             for (int kk = 0; kk < BKV / 16; ++kk) {
               const uint64_t db =
@@ -214,9 +224,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
           };
           bool ok = true;
           for (int j = 0; j < T && ok; ++j) {
-            const int s = j & 1;
-            const uint32_t ph = (j >> 1) & 1;
-            ok = ptx::mbar_wait(&k_full[s], ph, a.err, kErrTimeoutMma, abort_flag);
+            ok = ptx::mbar_wait(&k_full[j % K_STAGES], (j / K_STAGES) & 1, a.err, kErrTimeoutMma,
+                                abort_flag);
             if (!ok) break;
             ptx::tc_fence_after();
             issue_s(0, j);
@@ -226,11 +235,12 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
               if (!ok) break;
               ptx::tc_fence_after();
               issue_pv(1, j - 1);
-              ptx::mma_commit(&v_empty[(j - 1) & 1]);
+              ptx::mma_commit(&v_empty[(j - 1) % V_STAGES]);
             }
             issue_s(1, j);
-            ptx::mma_commit(&k_empty[s]);
-            ok = ptx::mbar_wait(&v_full[s], ph, a.err, kErrTimeoutMma, abort_flag);
+            ptx::mma_commit(&k_empty[j % K_STAGES]);
+            ok = ptx::mbar_wait(&v_full[j % V_STAGES], (j / V_STAGES) & 1, a.err, kErrTimeoutMma,
+                                abort_flag);
             if (ok) ok = ptx::mbar_wait(&p_full[0], j & 1, a.err, kErrTimeoutMma, abort_flag);
             if (!ok) break;
             ptx::tc_fence_after();
@@ -239,7 +249,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
           if (ok && ptx::mbar_wait(&p_full[1], (T - 1) & 1, a.err, kErrTimeoutMma, abort_flag)) {
             ptx::tc_fence_after();
             issue_pv(1, T - 1);
-            ptx::mma_commit(&v_empty[(T - 1) & 1]);
+            ptx::mma_commit(&v_empty[(T - 1) % V_STAGES]);
           }
         }
         ptx::mma_commit(mma_drain);
@@ -278,10 +288,17 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
         for (int i = 0; i < 128; ++i)
           if (key0 + i >= lim) sr[i] = __float_as_uint(-INFINITY);
       }
-      float mx = __uint_as_float(sr[0]);
+      // row max: four independent chains of 3-input maxima (a single chain is
+      // latency-bound), then combined
+      float m4[4];
 #pragma unroll
-      for (int i = 1; i < 127; i += 2) mx = fmax3(mx, __uint_as_float(sr[i]), __uint_as_float(sr[i + 1]));
-      mx = fmaxf(mx, __uint_as_float(sr[127]));
+      for (int q = 0; q < 4; ++q) m4[q] = fmaxf(__uint_as_float(sr[32 * q]), __uint_as_float(sr[32 * q + 1]));
+#pragma unroll
+      for (int i = 2; i < 32; i += 2)
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          m4[q] = fmax3(m4[q], __uint_as_float(sr[32 * q + i]), __uint_as_float(sr[32 * q + i + 1]));
+      const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
       const float m_tile = mx * sl2;
       const bool resc = m_tile > m_ref + kRescaleThreshold;
       float alpha = 1.f;
