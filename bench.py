@@ -225,12 +225,16 @@ def run_gpu(a):
         w = w.scaled(S_KV=a.s_kv)
     peaks = _peaks()
 
-    host = inputs.make(w, tensors=("q", "do", "y", "w_k", "w_v"))
-    pinned = {k: t.pin_memory() for k, t in host.items()}
-    d = {k: t.to(dev) for k, t in pinned.items()}
+    recompute = w.d_embed > 0   # K, V regenerated from y every step (else they are inputs)
+    host = inputs.make(w, tensors=("q", "do", "y", "w_k", "w_v") if recompute else ("q", "do", "k", "v"))
+    pinned = {k_: t.pin_memory() for k_, t in host.items()}
+    d = {k_: t.to(dev) for k_, t in pinned.items()}
     B, S_Q, H, hd = d["q"].shape
-    k = torch.empty(w.B, w.S_KV, w.H_kv, w.d, dtype=torch.bfloat16, device=dev)
-    v = torch.empty_like(k)
+    if recompute:
+        k = torch.empty(w.B, w.S_KV, w.H_kv, w.d, dtype=torch.bfloat16, device=dev)
+        v = torch.empty_like(k)
+    else:
+        k, v = d["k"], d["v"]
     out = torch.empty_like(d["q"])
     lse = torch.empty(B, H, S_Q, dtype=torch.float32, device=dev)
     dq = torch.empty_like(d["q"]); dk = torch.empty_like(k); dv = torch.empty_like(k)
@@ -240,11 +244,13 @@ def run_gpu(a):
 
     def step(ev=None):
         if ev: ev[0].record(stream)
-        lvx.lvx_kv_recompute(d["y"], d["w_k"], d["w_v"], k, v, w.H_kv, w.d)
+        if recompute:
+            lvx.lvx_kv_recompute(d["y"], d["w_k"], d["w_v"], k, v, w.H_kv, w.d)
         if ev: ev[1].record(stream)
         lvx.lvx_attn_fwd(d["q"], k, v, out, lse, w.n_blocks, w.causal, 0.0, fws)
         if ev: ev[2].record(stream)
-        lvx.lvx_attn_bwd(d["q"], k, v, out, lse, d["do"], dq, dk, dv, w.causal, 0.0, bws)
+        if w.backward:
+            lvx.lvx_attn_bwd(d["q"], k, v, out, lse, d["do"], dq, dk, dv, w.causal, 0.0, bws)
         if ev: ev[3].record(stream)
 
     warm = max(a.warmup, 3)
@@ -301,21 +307,28 @@ def run_gpu(a):
     # i+1 (copy stream) and the download of step i-1 (d2h stream) overlap the compute
     # of step i, with two device sets of inputs and outputs.  The timed region spans
     # the first upload through the last download.
-    res_host = {"dq": torch.empty(dq.shape, dtype=dq.dtype).pin_memory(),
-                "dk": torch.empty(dk.shape, dtype=dk.dtype).pin_memory(),
-                "dv": torch.empty(dv.shape, dtype=dv.dtype).pin_memory()}
+    res_names = ("dq", "dk", "dv") if w.backward else ("out",)
+    res_dev = {"dq": dq, "dk": dk, "dv": dv, "out": out}
+    res_host = {n_: torch.empty(res_dev[n_].shape, dtype=res_dev[n_].dtype).pin_memory()
+                for n_ in res_names}
     h2d = sum(t.numel() * t.element_size() for t in pinned.values())
     d2h = sum(t.numel() * t.element_size() for t in res_host.values())
     n_e2e = max(3, min(a.steps, 10))
     in_sets = [d, {k2: torch.empty_like(t) for k2, t in d.items()}]
-    out_sets = [{"dq": dq, "dk": dk, "dv": dv},
-                {"dq": torch.empty_like(dq), "dk": torch.empty_like(dk), "dv": torch.empty_like(dv)}]
+    out_sets = [{"dq": dq, "dk": dk, "dv": dv, "out": out, "lse": lse},
+                {"dq": torch.empty_like(dq), "dk": torch.empty_like(dk), "dv": torch.empty_like(dv),
+                 "out": torch.empty_like(out), "lse": torch.empty_like(lse)}]
 
     def run_step(inp, o):
-        lvx.lvx_kv_recompute(inp["y"], inp["w_k"], inp["w_v"], k, v, w.H_kv, w.d)
-        lvx.lvx_attn_fwd(inp["q"], k, v, out, lse, w.n_blocks, w.causal, 0.0, fws)
-        lvx.lvx_attn_bwd(inp["q"], k, v, out, lse, inp["do"], o["dq"], o["dk"], o["dv"], w.causal,
-                         0.0, bws)
+        kk, vv = k, v
+        if recompute:
+            lvx.lvx_kv_recompute(inp["y"], inp["w_k"], inp["w_v"], k, v, w.H_kv, w.d)
+        else:
+            kk, vv = inp["k"], inp["v"]
+        lvx.lvx_attn_fwd(inp["q"], kk, vv, o["out"], o["lse"], w.n_blocks, w.causal, 0.0, fws)
+        if w.backward:
+            lvx.lvx_attn_bwd(inp["q"], kk, vv, o["out"], o["lse"], inp["do"], o["dq"], o["dk"],
+                             o["dv"], w.causal, 0.0, bws)
 
     copy_s, d2h_s = torch.cuda.Stream(), torch.cuda.Stream()
     ev = lambda: torch.cuda.Event()
@@ -348,7 +361,7 @@ def run_gpu(a):
         out_done[cur].record(stream)
         with torch.cuda.stream(d2h_s):
             d2h_s.wait_event(out_done[cur])
-            for name in ("dq", "dk", "dv"):
+            for name in res_names:
                 res_host[name].copy_(out_sets[cur][name], non_blocking=True)
             out_free[cur].record(d2h_s)
     stream.wait_stream(d2h_s)
@@ -363,14 +376,16 @@ def run_gpu(a):
     stages = {"bwd": (t_bwd, w.bwd_flops(), "lvx_attn_bwd (preprocess + main + dQ finalize)"),
               "fwd": (t_fwd, w.fwd_flops(), "lvx_attn_fwd (block partials + merge)"),
               "kv": (t_kv, w.kv_flops(), "lvx_kv_recompute")}
+    stages = {k_: v_ for k_, v_ in stages.items() if v_[1] > 0}
     dom = max(stages, key=lambda s: stages[s][0])
     t_dom, f_dom, dom_desc = stages[dom]
     achieved = f_dom / (t_dom * 1e-3) / 1e12
     tr = TRAFFIC.get(dom)
     traffic = tr["bytes"] if tr and _file_sha(tr["source"]) == tr["sha"] else None
-    # kv recompute, fwd partials, merge, bwd preprocess, bwd main, dQ finalize (this workload
-    # takes the tensor-core kernels: one launch each)
-    launches_per_step = 6
+    # tensor-core dispatch: K/V recompute (1), fwd partials (1) + merge (n_blocks > 1),
+    # bwd preprocess + main + dQ finalize (3)
+    launches_per_step = (1 if recompute else 0) + 1 + (1 if w.n_blocks > 1 else 0) + \
+        (3 if w.backward else 0)
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": a.steps,
         "warmup": warm, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -379,8 +394,8 @@ def run_gpu(a):
         "config": _config(w, world),
         "pct_of_peak": 100.0 * value / peaks["bf16_sust"],
         "stages_ms": {"kv_recompute": t_kv, "fwd": t_fwd, "bwd": t_bwd},
-        "stage_tflops": {s: (stages[s][1] / (stages[s][0] * 1e-3) / 1e12 if stages[s][0] else None)
-                         for s in stages},
+        "stage_tflops": {s_: (stages[s_][1] / (stages[s_][0] * 1e-3) / 1e12 if stages[s_][0] else None)
+                         for s_ in stages},
         "roofline": {"bound": "tensor", "kernel": dom_desc, "achieved": achieved,
                      "peak": peaks["bf16_sust"], "unit": "TFLOP/s",
                      "frac": achieved / peaks["bf16_sust"], "traffic": traffic,
