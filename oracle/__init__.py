@@ -19,7 +19,7 @@ The oracle is written from these pages:
   exact), the referee report's first major comment (the backward pass is
   not specified; checked here against the exact formula's gradient), and
   Figure 1 / the activation-recomputation passage (K = y W_k, V = y W_v from
-  one shared copy of the visual features y).
+  one shared copy of the visual features y, and the gradients of that map).
 
 Every function is pinned by tests under ``tests/`` against closed forms,
 invariants, brute force on tiny inputs and an independent library routine
@@ -37,4 +37,5 @@ from .attention import (  # noqa: F401
     attention_bwd_keys,
     attention_bwd_rows,
     kv_recompute,
+    kv_recompute_bwd,
 )

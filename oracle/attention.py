@@ -296,3 +296,29 @@ def kv_recompute(y, w_k, w_v, rows: Optional[Sequence[int]] = None):
     if rows is not None:
         y = y[..., np.asarray(rows), :]
     return y @ w_k, y @ w_v
+
+
+def kv_recompute_bwd(y, w_k, w_v, dk, dv, rows: Optional[Sequence[int]] = None):
+    """Gradients of the K/V recomputation K = y W_k, V = y W_v.
+
+    LV-XAttn review page, "What carries the argument" and Figure 6: keys and
+    values are regenerated from the one shared copy of the visual features
+    y, so training needs the gradients of that linear map (the pages do not
+    write them out; this is the textbook gradient of a matrix product):
+      dW_k = y^T dK,   dW_v = y^T dV,   dy = dK W_k^T + dV W_v^T.
+    y [S, d_embed] (or [B, S, d_embed], batches summed into dW); dk, dv
+    [..., S, H_kv*d]; ``rows`` restricts dy to some rows (dW always uses all).
+    Returns dy, dw_k, dw_v in fp64.
+    """
+    y = _f64(y); w_k = _f64(w_k); w_v = _f64(w_v); dk = _f64(dk); dv = _f64(dv)
+    y2 = y.reshape(-1, y.shape[-1])
+    dk2 = dk.reshape(-1, dk.shape[-1])
+    dv2 = dv.reshape(-1, dv.shape[-1])
+    dw_k = y2.T @ dk2
+    dw_v = y2.T @ dv2
+    if rows is not None:
+        rows = np.asarray(rows)
+        dy = dk[..., rows, :] @ w_k.T + dv[..., rows, :] @ w_v.T
+    else:
+        dy = dk @ w_k.T + dv @ w_v.T
+    return dy, dw_k, dw_v

@@ -319,6 +319,50 @@ def test_kv_recompute_exact_on_integers():
     np.testing.assert_array_equal(Ks, K[:, [1, 4]])
 
 
+def test_kv_recompute_bwd_matches_central_differences():
+    rng = np.random.default_rng(17)
+    y = rng.standard_normal((6, 5)); wk = rng.standard_normal((5, 4)); wv = rng.standard_normal((5, 4))
+    dk = rng.standard_normal((6, 4)); dv = rng.standard_normal((6, 4))
+    dy, dwk, dwv = oracle.kv_recompute_bwd(y, wk, wv, dk, dv)
+
+    def f(y_, wk_, wv_):
+        K, V = oracle.kv_recompute(y_, wk_, wv_)
+        return float((K * dk).sum() + (V * dv).sum())
+
+    eps = 1e-6
+    for x, g, name in ((y, dy, "y"), (wk, dwk, "wk"), (wv, dwv, "wv")):
+        num = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            xp = x.copy(); xp[idx] += eps
+            xm = x.copy(); xm[idx] -= eps
+            args = {"y": y, "wk": wk, "wv": wv}
+            args[name] = xp; fp = f(args["y"], args["wk"], args["wv"])
+            args[name] = xm; fm = f(args["y"], args["wk"], args["wv"])
+            num[idx] = (fp - fm) / (2 * eps)
+        np.testing.assert_allclose(num, g, rtol=1e-7, atol=1e-7)
+
+
+def test_kv_recompute_bwd_exact_on_integers_and_batches():
+    rng = np.random.default_rng(18)
+    y = rng.integers(-3, 4, size=(2, 5, 6)).astype(np.float64)
+    wk = rng.integers(-2, 3, size=(6, 4)).astype(np.float64)
+    wv = rng.integers(-2, 3, size=(6, 4)).astype(np.float64)
+    dk = rng.integers(-2, 3, size=(2, 5, 4)).astype(np.float64)
+    dv = rng.integers(-2, 3, size=(2, 5, 4)).astype(np.float64)
+    dy, dwk, dwv = oracle.kv_recompute_bwd(y, wk, wv, dk, dv)
+    for e in range(6):
+        for c in range(4):
+            assert dwk[e, c] == sum(int(y[b, s, e]) * int(dk[b, s, c]) for b in range(2) for s in range(5))
+            assert dwv[e, c] == sum(int(y[b, s, e]) * int(dv[b, s, c]) for b in range(2) for s in range(5))
+    for b in range(2):
+        for s in range(5):
+            for e in range(6):
+                assert dy[b, s, e] == sum(int(dk[b, s, c]) * int(wk[e, c]) + int(dv[b, s, c]) * int(wv[e, c])
+                                          for c in range(4))
+    dys, _, _ = oracle.kv_recompute_bwd(y, wk, wv, dk, dv, rows=[0, 3])
+    np.testing.assert_array_equal(dys, dy[:, [0, 3]])
+
+
 # ---------------------------------------------------------------- planted mistakes
 
 def _pins_fail(monkeypatch, name, bad):
