@@ -111,12 +111,13 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- CPU oracle baseline
 
-def oracle_sample(w, seconds_hint: float = 20.0):
+def oracle_sample(w, kv_grads: bool = False):
     """Times the fp64 oracle on a bounded sample of the workload's step.
 
     Sample: the same heads, head width and S_KV, with S_Q cut to ``rows``
     query rows (forward + full textbook backward), plus K/V recomputation of
-    ``rows`` rows of y.  Returns (TFLOP/s of counted work, seconds, description).
+    ``rows`` rows of y (and, with ``kv_grads``, its gradients over those rows).
+    Returns (TFLOP/s of counted work, seconds, description).
     """
     import numpy as np
     import oracle
@@ -139,9 +140,15 @@ def oracle_sample(w, seconds_hint: float = 20.0):
         y = np.random.default_rng(0).standard_normal((rows, w.d_embed))
         oracle.kv_recompute(y, kvw["w_k"].double().numpy(), kvw["w_v"].double().numpy())
         flops += 2 * 2 * rows * w.d_embed * w.H_kv * w.d
+        if kv_grads:
+            g = np.random.default_rng(1).standard_normal((2, rows, w.H_kv * w.d))
+            oracle.kv_recompute_bwd(y, kvw["w_k"].double().numpy(), kvw["w_v"].double().numpy(),
+                                    g[0], g[1])
+            flops += 2 * 2 * 2 * rows * w.d_embed * w.H_kv * w.d
     dt = time.perf_counter() - t0
     desc = (f"fp64 oracle, forward + backward for {rows} of {w.S_Q} query rows over all {w.H} heads "
-            f"and all {w.S_KV} keys, plus K/V recompute of {rows} rows of y; counted FLOPs / time")
+            f"and all {w.S_KV} keys, plus K/V recompute of {rows} rows of y"
+            f"{' and its gradients' if kv_grads and kvw is not None else ''}; counted FLOPs / time")
     return flops / dt / 1e12, dt, cores, desc
 
 
@@ -151,19 +158,20 @@ def run_reference(a):
         return
     from blockwise_long_context_b200 import inputs
     w = inputs.WORKLOADS[a.workload]
+    kv_grads = a.kv_grads and w.d_embed > 0 and w.backward
     for _ in range(a.warmup):
-        oracle_sample(w)
+        oracle_sample(w, kv_grads)
     vals, secs = [], []
     cores, desc = 1, ""
     for _ in range(a.steps):
-        v, s, cores, desc = oracle_sample(w)
+        v, s, cores, desc = oracle_sample(w, kv_grads)
         vals.append(v); secs.append(s)
     value = statistics.mean(vals)
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": a.gpus,
             "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * statistics.mean(secs),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
-            "config": _config(w, a.gpus),
+            "config": _config(w, a.gpus, kv_grads),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                              "sample": desc},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -171,13 +179,17 @@ def run_reference(a):
     print(json.dumps(line), flush=True)
 
 
-def _config(w, n):
-    return {"workload": f"{w.name}: {w.desc}", "B": w.B, "H": w.H, "H_kv": w.H_kv, "d": w.d,
-            "S_Q": w.S_Q, "S_KV": w.S_KV, "n_blocks": w.n_blocks, "causal": w.causal,
-            "d_embed": w.d_embed, "parallelism": f"replicas{n}" if n > 1 else "single",
-            "l2": "inputs larger than L2: y 512 MiB read and K/V 256 MiB rewritten every step",
-            "flops_counted": "attn fwd 4*B*H*S_Q*S_KV*d + bwd 2.5x fwd + K/V recompute "
-                             "2*2*B*S_KV*d_embed*H_kv*d"}
+def _config(w, n, kv_grads=False):
+    c = {"workload": f"{w.name}: {w.desc}", "B": w.B, "H": w.H, "H_kv": w.H_kv, "d": w.d,
+         "S_Q": w.S_Q, "S_KV": w.S_KV, "n_blocks": w.n_blocks, "causal": w.causal,
+         "d_embed": w.d_embed, "parallelism": f"replicas{n}" if n > 1 else "single",
+         "l2": "inputs larger than L2: y 512 MiB read and K/V 256 MiB rewritten every step",
+         "flops_counted": "attn fwd 4*B*H*S_Q*S_KV*d + bwd 2.5x fwd + K/V recompute "
+                          "2*2*B*S_KV*d_embed*H_kv*d"}
+    if kv_grads:
+        c["kv_grads"] = True
+        c["flops_counted"] += " + its gradients dW_k, dW_v, dy 2x the recompute"
+    return c
 
 
 # ---------------------------------------------------------------- multi-rank helpers
@@ -226,6 +238,7 @@ def run_gpu(a):
     peaks = _peaks()
 
     recompute = w.d_embed > 0   # K, V regenerated from y every step (else they are inputs)
+    kv_grads = recompute and w.backward and a.kv_grads   # + dW_k, dW_v, dy of the recomputation
     host = inputs.make(w, tensors=("q", "do", "y", "w_k", "w_v") if recompute else ("q", "do", "k", "v"))
     pinned = {k_: t.pin_memory() for k_, t in host.items()}
     d = {k_: t.to(dev) for k_, t in pinned.items()}
@@ -238,6 +251,8 @@ def run_gpu(a):
     out = torch.empty_like(d["q"])
     lse = torch.empty(B, H, S_Q, dtype=torch.float32, device=dev)
     dq = torch.empty_like(d["q"]); dk = torch.empty_like(k); dv = torch.empty_like(k)
+    if kv_grads:
+        dy = torch.empty_like(d["y"]); dwk = torch.empty_like(d["w_k"]); dwv = torch.empty_like(d["w_v"])
     fws = lvx.fwd_workspace(d["q"], k, w.n_blocks, w.causal)
     bws = lvx.bwd_workspace(d["q"], k, w.causal)
     stream = torch.cuda.current_stream()
@@ -252,6 +267,9 @@ def run_gpu(a):
         if w.backward:
             lvx.lvx_attn_bwd(d["q"], k, v, out, lse, d["do"], dq, dk, dv, w.causal, 0.0, bws)
         if ev: ev[3].record(stream)
+        if kv_grads:
+            lvx.lvx_kv_recompute_bwd(d["y"], d["w_k"], d["w_v"], dk, dv, dy, dwk, dwv)
+        if ev: ev[4].record(stream)
 
     warm = max(a.warmup, 3)
     for _ in range(warm):
@@ -259,7 +277,7 @@ def run_gpu(a):
     torch.cuda.synchronize()
     lvx.lvx_last_device_error()
 
-    stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(a.steps)]
+    stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(a.steps)]
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local)
     if world > 1:
@@ -279,11 +297,13 @@ def run_gpu(a):
     t_kv = statistics.mean(ev[0].elapsed_time(ev[1]) for ev in stage_ev)
     t_fwd = statistics.mean(ev[1].elapsed_time(ev[2]) for ev in stage_ev)
     t_bwd = statistics.mean(ev[2].elapsed_time(ev[3]) for ev in stage_ev)
+    t_kvb = statistics.mean(ev[3].elapsed_time(ev[4]) for ev in stage_ev)
     lvx.lvx_last_device_error()
 
     ms_total = max_over_ranks(ms_total, dev)
     ms_step = ms_total / a.steps
-    step_flops = w.fwd_flops() + w.bwd_flops() + w.kv_flops()
+    kvb_flops = 2.0 * w.kv_flops() if kv_grads else 0.0
+    step_flops = w.fwd_flops() + w.bwd_flops() + w.kv_flops() + kvb_flops
     value = whole_job_tflops(step_flops, a.steps, world, ms_total)
 
     # merge kernel alone (HBM-bound), after an L2 flush, through the merge entry point
@@ -309,6 +329,9 @@ def run_gpu(a):
     # the first upload through the last download.
     res_names = ("dq", "dk", "dv") if w.backward else ("out",)
     res_dev = {"dq": dq, "dk": dk, "dv": dv, "out": out}
+    if kv_grads:   # the gradients reaching y and the weights replace dK, dV as results
+        res_names = ("dq", "dy", "dwk", "dwv")
+        res_dev.update(dy=dy, dwk=dwk, dwv=dwv)
     res_host = {n_: torch.empty(res_dev[n_].shape, dtype=res_dev[n_].dtype).pin_memory()
                 for n_ in res_names}
     h2d = sum(t.numel() * t.element_size() for t in pinned.values())
@@ -318,6 +341,10 @@ def run_gpu(a):
     out_sets = [{"dq": dq, "dk": dk, "dv": dv, "out": out, "lse": lse},
                 {"dq": torch.empty_like(dq), "dk": torch.empty_like(dk), "dv": torch.empty_like(dv),
                  "out": torch.empty_like(out), "lse": torch.empty_like(lse)}]
+    if kv_grads:
+        out_sets[0].update(dy=dy, dwk=dwk, dwv=dwv)
+        out_sets[1].update(dy=torch.empty_like(dy), dwk=torch.empty_like(dwk),
+                           dwv=torch.empty_like(dwv))
 
     def run_step(inp, o):
         kk, vv = k, v
@@ -329,6 +356,9 @@ def run_gpu(a):
         if w.backward:
             lvx.lvx_attn_bwd(inp["q"], kk, vv, o["out"], o["lse"], inp["do"], o["dq"], o["dk"],
                              o["dv"], w.causal, 0.0, bws)
+        if kv_grads:
+            lvx.lvx_kv_recompute_bwd(inp["y"], inp["w_k"], inp["w_v"], o["dk"], o["dv"], o["dy"],
+                                     o["dwk"], o["dwv"])
 
     copy_s, d2h_s = torch.cuda.Stream(), torch.cuda.Stream()
     ev = lambda: torch.cuda.Event()
@@ -375,7 +405,8 @@ def run_gpu(a):
     # roofline of the dominant kernel group (timed inside the long step loop: sustained peak)
     stages = {"bwd": (t_bwd, w.bwd_flops(), "lvx_attn_bwd (preprocess + main + dQ finalize)"),
               "fwd": (t_fwd, w.fwd_flops(), "lvx_attn_fwd (block partials + merge)"),
-              "kv": (t_kv, w.kv_flops(), "lvx_kv_recompute")}
+              "kv": (t_kv, w.kv_flops(), "lvx_kv_recompute"),
+              "kv_bwd": (t_kvb, kvb_flops, "lvx_kv_recompute_bwd")}
     stages = {k_: v_ for k_, v_ in stages.items() if v_[1] > 0}
     dom = max(stages, key=lambda s: stages[s][0])
     t_dom, f_dom, dom_desc = stages[dom]
@@ -385,15 +416,16 @@ def run_gpu(a):
     # tensor-core dispatch: K/V recompute (1), fwd partials (1) + merge (n_blocks > 1),
     # bwd preprocess + main + dQ finalize (3)
     launches_per_step = (1 if recompute else 0) + 1 + (1 if w.n_blocks > 1 else 0) + \
-        (3 if w.backward else 0)
+        (3 if w.backward else 0) + (2 if kv_grads else 0)
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": a.steps,
         "warmup": warm, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded Gaussian, shapes of the "
         "pages' Llama-3-V cross-attention workload)",
-        "config": _config(w, world),
+        "config": _config(w, world, kv_grads),
         "pct_of_peak": 100.0 * value / peaks["bf16_sust"],
-        "stages_ms": {"kv_recompute": t_kv, "fwd": t_fwd, "bwd": t_bwd},
+        "stages_ms": {"kv_recompute": t_kv, "fwd": t_fwd, "bwd": t_bwd,
+                      **({"kv_recompute_bwd": t_kvb} if kv_grads else {})},
         "stage_tflops": {s_: (stages[s_][1] / (stages[s_][0] * 1e-3) / 1e12 if stages[s_][0] else None)
                          for s_ in stages},
         "roofline": {"bound": "tensor", "kernel": dom_desc, "achieved": achieved,
@@ -409,7 +441,7 @@ def run_gpu(a):
         "clocks": clk,
     }
     if world == 1 and rank == 0 and not a.no_cpu_baseline:
-        cv, cs, cores, desc = oracle_sample(w)
+        cv, cs, cores, desc = oracle_sample(w, kv_grads)
         line["cpu_baseline"] = {"value": cv, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                                 "sample": desc, "seconds": cs}
     if rank == 0:
@@ -427,6 +459,8 @@ def main():
     ap.add_argument("--impl", default="lvx", choices=["lvx", "reference"])
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kv-grads", action="store_true",
+                    help="also run the gradients of the K/V recomputation (dW_k, dW_v, dy) each step")
     ap.add_argument("--s-kv", type=int, default=0,
                     help="override S_KV (smaller case of the same workload, for profiler captures)")
     a = ap.parse_args()

@@ -14,7 +14,7 @@ every call raises.
 from __future__ import annotations
 
 __all__ = [
-    "LvxError", "lib", "lvx_attn_fwd", "lvx_attn_bwd", "lvx_kv_recompute",
+    "LvxError", "lib", "lvx_attn_fwd", "lvx_attn_bwd", "lvx_kv_recompute", "lvx_kv_recompute_bwd",
     "lvx_merge_partials", "lvx_attn_fwd_noalloc", "lvx_attn_fwd_workspace", "lvx_attn_bwd_workspace",
     "lvx_last_device_error", "lvx_status_string", "LVX_FP32", "LVX_BF16",
 ]

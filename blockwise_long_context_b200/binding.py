@@ -43,6 +43,7 @@ _SIGS = {
     "lvx_attn_bwd_workspace": ([_c_int] * 7 + [_c_int], _c_size),
     "lvx_attn_bwd": ([_vp] * 9 + [_c_int] * 7 + [_c_int, _c_float, _vp, _c_size, _vp], _c_int),
     "lvx_kv_recompute": ([_vp] * 5 + [_c_int] * 5 + [_c_int, _vp], _c_int),
+    "lvx_kv_recompute_bwd": ([_vp] * 8 + [_c_int] * 5 + [_c_int, _vp], _c_int),
     "lvx_last_device_error": ([_vp], _c_int),
     "lvx_selftest_wait_timeout": ([_vp], _c_int),
 }
@@ -150,6 +151,16 @@ def lvx_kv_recompute(y, w_k, w_v, k, v, H_kv: int, d: int, stream=None) -> None:
                                   d_embed, H_kv, d, _dt(y), _stream(stream)), "lvx_kv_recompute")
 
 
+def lvx_kv_recompute_bwd(y, w_k, w_v, dk, dv, dy, dw_k, dw_v, stream=None) -> None:
+    """y [B,S_KV,d_embed], w [d_embed,H_kv*d], dk/dv [B,S_KV,H_kv,d] ->
+    dy like y, dw_k/dw_v like w (dW = y^T dK, dy = dK W_k^T + dV W_v^T)."""
+    B, S_KV, d_embed = y.shape
+    H_kv, d = dk.shape[2], dk.shape[3]
+    _check(lib().lvx_kv_recompute_bwd(_ptr(y), _ptr(w_k), _ptr(w_v), _ptr(dk), _ptr(dv), _ptr(dy),
+                                      _ptr(dw_k), _ptr(dw_v), B, S_KV, d_embed, H_kv, d, _dt(y),
+                                      _stream(stream)), "lvx_kv_recompute_bwd")
+
+
 def lvx_last_device_error(stream=None) -> None:
     _check(lib().lvx_last_device_error(_stream(stream)), "lvx_last_device_error")
 
@@ -192,6 +203,13 @@ def attention_forward(q, k, v, n_blocks: int, causal: bool = False, scale: float
     ws = fwd_workspace(q, k, n_blocks, causal)
     lvx_attn_fwd(q, k, v, out, lse, n_blocks, causal, scale, ws)
     return out, lse
+
+
+def kv_recompute_backward(y, w_k, w_v, dk, dv):
+    """Allocates dy, dw_k, dw_v and runs lvx_kv_recompute_bwd; returns them."""
+    dy = torch.empty_like(y); dw_k = torch.empty_like(w_k); dw_v = torch.empty_like(w_v)
+    lvx_kv_recompute_bwd(y, w_k, w_v, dk, dv, dy, dw_k, dw_v)
+    return dy, dw_k, dw_v
 
 
 def attention_backward(q, k, v, out, lse, dout, causal: bool = False, scale: float = 0.0):

@@ -183,8 +183,47 @@ lvx_status lvx_kv_recompute(const void* y, const void* w_k, const void* w_v, voi
   if (dt == LVX_BF16 && tc_gemm_supported(M, K, N)) {
     e = launch_kv_gemm_tc(y, w_k, w_v, k, v, M, K, N, s);
   } else {
-    e = launch_gemm_simt(y, w_k, k, M, K, N, dt, s);
-    if (e == cudaSuccess) e = launch_gemm_simt(y, w_v, v, M, K, N, dt, s);
+    // K = y W_k, V = y W_v: A = y (row stride K), B = W (row stride N)
+    SimtGemm g{{y, nullptr}, {w_k, nullptr}, k, (size_t)K, 1, (size_t)N, 1, M, N, K, 1};
+    e = launch_gemm_simt(g, dt, s);
+    if (e == cudaSuccess) {
+      g.B[0] = w_v;
+      g.C = v;
+      e = launch_gemm_simt(g, dt, s);
+    }
+  }
+  return from_cuda(e);
+}
+
+lvx_status lvx_kv_recompute_bwd(const void* y, const void* w_k, const void* w_v, const void* dk,
+                                const void* dv, void* dy, void* dw_k, void* dw_v, int B, int S_KV,
+                                int d_embed, int H_kv, int d, lvx_dtype dt, lvx_stream stream) {
+  if (B < 1 || S_KV < 1 || d_embed < 1 || H_kv < 1 || d < 1) return LVX_ERR_INVALID_ARG;
+  if (dt != LVX_FP32 && dt != LVX_BF16) return LVX_ERR_UNSUPPORTED;
+  const void* ptrs[] = {y, w_k, w_v, dk, dv, dy, dw_k, dw_v};
+  for (const void* ptr : ptrs)
+    if (!ptr || !aligned16(ptr)) return LVX_ERR_INVALID_ARG;
+  if ((long long)B * S_KV > (1ll << 31) - 1 || (long long)H_kv * d > (1 << 30))
+    return LVX_ERR_UNSUPPORTED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int S = B * S_KV, E = d_embed, N = H_kv * d;
+  cudaError_t e;
+  if (dt == LVX_BF16 && tc_gemm_bwd_supported(S, E, N)) {
+    e = launch_kv_gemm_bwd_tc(y, w_k, w_v, dk, dv, dy, dw_k, dw_v, S, E, N, s);
+  } else {
+    // dW_k = y^T dK: A(m=e, k=s) = y[s][e], B(k=s, n) = dK[s][n]
+    SimtGemm g{{y, nullptr}, {dk, nullptr}, dw_k, 1, (size_t)E, (size_t)N, 1, E, N, S, 1};
+    e = launch_gemm_simt(g, dt, s);
+    if (e == cudaSuccess) {
+      g.B[0] = dv;
+      g.C = dw_v;
+      e = launch_gemm_simt(g, dt, s);
+    }
+    if (e == cudaSuccess) {
+      // dy = dK W_k^T + dV W_v^T: A(m=s, k=n) = dZ[s][n], B(k=n, n'=e) = W_z[e][n]
+      SimtGemm h{{dk, dv}, {w_k, w_v}, dy, (size_t)N, 1, 1, (size_t)N, S, E, N, 2};
+      e = launch_gemm_simt(h, dt, s);
+    }
   }
   return from_cuda(e);
 }

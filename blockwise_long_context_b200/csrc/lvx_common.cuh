@@ -70,7 +70,16 @@ cudaError_t launch_bwd_simt(const Problem& p, lvx_dtype dt, const void* q, const
                             float* dq_acc, void* dk, void* dv, cudaStream_t s);
 cudaError_t launch_dq_finalize(const float* dq_acc, void* dq, size_t count, float scale,
                                lvx_dtype dt, cudaStream_t s);
-cudaError_t launch_gemm_simt(const void* y, const void* w, void* out, int M, int K, int N,
-                             lvx_dtype dt, cudaStream_t s);
+// C [M][N] row-major = sum over `segments` (1 or 2) of A_g B_g, where element
+// (m, k) of A_g is A[g][m*sam + k*sak] and element (k, n) of B_g is
+// B[g][k*sbk + n*sbn]; every segment has the same K.
+struct SimtGemm {
+  const void* A[2];
+  const void* B[2];
+  void* C;
+  size_t sam, sak, sbk, sbn;
+  int M, N, K, segments;
+};
+cudaError_t launch_gemm_simt(const SimtGemm& g, lvx_dtype dt, cudaStream_t s);
 
 }  // namespace lvx

@@ -1,13 +1,19 @@
-// K/V recomputation from the shared visual features on the tcgen05 tensor
-// cores: K = y W_k and V = y W_v in one launch (LV-XAttn review page,
-// "What carries the argument" and Figure 6: one copy of y is kept and the
-// keys/values are regenerated from it).
-//
-// Tile: 128 rows of y x 256 output columns, K step 64.  TMA brings the y tile
-// (K-major, 128-byte swizzle) and four 64x64 boxes of W (N-major, 128-byte
-// swizzle) into a 4-stage ring; one thread issues tcgen05.mma (M=128, N=256,
-// K=16) into a 256-column fp32 TMEM accumulator; the four warps then read
-// the accumulator (one 32-lane quarter each), round to bf16 and store.
+// K/V recomputation from the shared visual features and its gradients on
+// the tcgen05 tensor cores (LV-XAttn review page, "What carries the argument"
+// and Figure 6: one copy of the visual features y is kept and the keys and
+// values are regenerated from it; training needs the gradients of that map).
+//   forward:   K = y W_k,  V = y W_v                 (A = y K-major, B = W N-major)
+//   gradient:  dW_k = y^T dK,  dW_v = y^T dV          (A = y M-major, B = dK N-major)
+//              dy = dK W_k^T + dV W_v^T               (A = dK K-major, B = W K-major,
+//                                                      two K segments summed)
+// One kernel template serves all three: tile 128 x 256 outputs, K step 64,
+// a 4-stage TMA ring (128-byte swizzle; K-major tiles are 64-element rows
+// along K, M/N-major tiles are 64-element rows along M/N), one thread
+// issuing tcgen05.mma (M=128, N=256, K=16) into a 256-column fp32 TMEM
+// accumulator, and four warps reading it back (one 32-lane quarter each),
+// rounding to bf16 and storing.  In batched mode a launch holds two
+// independent problems (forward K and V, or dW_k and dW_v); in segment mode a
+// single problem's K loop runs over two (A, B) pairs.
 #include "lvx_ptx.cuh"
 #include "lvx_tc.cuh"
 
@@ -16,22 +22,25 @@ namespace {
 
 constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
 constexpr uint32_t A_BYTES = BM * BK * 2;          // 16 KiB
-constexpr uint32_t B_BOX_BYTES = BK * 64 * 2;      // 8 KiB: 64 K-rows x 64 N
-constexpr uint32_t B_BYTES = 4 * B_BOX_BYTES;      // 32 KiB
+constexpr uint32_t B_BYTES = BN * BK * 2;          // 32 KiB
 constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr uint32_t SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
-constexpr uint32_t IDESC = ptx::idesc_bf16_f32(BM, BN, false, true);
 
 struct GemmArgs {
-  __nv_bfloat16* out_k;
-  __nv_bfloat16* out_v;
+  __nv_bfloat16* out[2];   // [M][N] row-major, per problem
   unsigned int* err;
-  int M, K, N;   // N = columns of each weight
+  int M, N;
+  int kb_seg0;             // k-blocks taken from (A0, B0); the rest from (A1, B1)
+  int kb_total;            // k-blocks per output tile
+  int batched;             // 1: two problems (A_z, B_z) -> out[z]; 0: two K segments -> out[0]
 };
 
+template <bool A_MN, bool B_MN>
 __global__ void __launch_bounds__(128, 1)
-kv_gemm_kernel(const __grid_constant__ CUtensorMap map_y, const __grid_constant__ CUtensorMap map_wk,
-               const __grid_constant__ CUtensorMap map_wv, GemmArgs args) {
+gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a0, const __grid_constant__ CUtensorMap map_b0,
+               const __grid_constant__ CUtensorMap map_a1, const __grid_constant__ CUtensorMap map_b1,
+               GemmArgs args) {
+  constexpr uint32_t IDESC = ptx::idesc_bf16_f32(BM, BN, A_MN, B_MN);
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -42,12 +51,14 @@ kv_gemm_kernel(const __grid_constant__ CUtensorMap map_y, const __grid_constant_
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_tiles_per_w = args.N / BN;
-  const bool is_v = blockIdx.x >= n_tiles_per_w;
-  const int n0 = (blockIdx.x % n_tiles_per_w) * BN;
-  const int m0 = blockIdx.y * BM;
-  const int kblocks = args.K / BK;
-  const CUtensorMap* map_w = is_v ? &map_wv : &map_wk;
+  // Tile order: N tiles fastest, then the problem, then M, so that the CTAs
+  // resident together share their A tile (and, when batched, A is the same
+  // matrix y for both problems) and it is read from HBM about once.
+  const int n_tiles = args.N / BN;
+  const int problems = args.batched ? 2 : 1;
+  const int n0 = (int)(blockIdx.x % n_tiles) * BN;
+  const int z = (int)(blockIdx.x / n_tiles) % problems;
+  const int m0 = (int)(blockIdx.x / (n_tiles * problems)) * BM;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -59,8 +70,12 @@ kv_gemm_kernel(const __grid_constant__ CUtensorMap map_y, const __grid_constant_
     ptx::fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
-    ptx::tma_prefetch_desc(&map_y);
-    ptx::tma_prefetch_desc(map_w);
+    ptx::tma_prefetch_desc(args.batched && z ? &map_a1 : &map_a0);
+    ptx::tma_prefetch_desc(args.batched && z ? &map_b1 : &map_b0);
+    if (!args.batched) {
+      ptx::tma_prefetch_desc(&map_a1);
+      ptx::tma_prefetch_desc(&map_b1);
+    }
   }
   if (warp == 2) {
     ptx::tmem_alloc(tmem_slot, BN);
@@ -72,19 +87,31 @@ kv_gemm_kernel(const __grid_constant__ CUtensorMap map_y, const __grid_constant_
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0 && lane == 0) {
-    // producer
+    // ------------------------------------------------------------------ producer
     int issued = 0;
-    for (int kb = 0; kb < kblocks; ++kb) {
+    for (int kb = 0; kb < args.kb_total; ++kb) {
       const int s = kb % STAGES;
       const uint32_t round = kb / STAGES;
       if (!ptx::mbar_wait(&empty[s], (round & 1) ^ 1, args.err, kErrTimeoutTma, abort_flag)) break;
+      const bool second = z == 1 || kb >= args.kb_seg0;
+      const CUtensorMap* ma = second ? &map_a1 : &map_a0;
+      const CUtensorMap* mb = second ? &map_b1 : &map_b0;
+      const int k0 = (kb >= args.kb_seg0 && !args.batched ? kb - args.kb_seg0 : kb) * BK;
       uint8_t* a = smem + s * STAGE_BYTES;
       uint8_t* b = a + A_BYTES;
       ptx::mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
-      ptx::tma_load_2d(a, &map_y, &full[s], kb * BK, m0);
+      if (A_MN) {   // A stored [K][M]: two 64-wide M chunks of 64 K rows
+        ptx::tma_load_2d(a, ma, &full[s], m0, k0);
+        ptx::tma_load_2d(a + 8192, ma, &full[s], m0 + 64, k0);
+      } else {      // A stored [M][K]: 128 rows of 64 K
+        ptx::tma_load_2d(a, ma, &full[s], k0, m0);
+      }
+      if (B_MN) {   // B stored [K][N]: four 64-wide N chunks of 64 K rows
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
-        ptx::tma_load_2d(b + j * B_BOX_BYTES, map_w, &full[s], n0 + 64 * j, kb * BK);
+        for (int j = 0; j < 4; ++j) ptx::tma_load_2d(b + j * 8192, mb, &full[s], n0 + 64 * j, k0);
+      } else {      // B stored [N][K]: 256 rows of 64 K
+        ptx::tma_load_2d(b, mb, &full[s], k0, n0);
+      }
       issued = kb + 1;
     }
     if (*abort_flag) {
@@ -93,8 +120,8 @@ kv_gemm_kernel(const __grid_constant__ CUtensorMap map_y, const __grid_constant_
         ptx::mbar_wait(&full[kb % STAGES], (kb / STAGES) & 1, args.err, kErrTimeoutTma, nullptr);
     }
   } else if (warp == 1 && lane == 0) {
-    // MMA issuer
-    for (int kb = 0; kb < kblocks; ++kb) {
+    // ------------------------------------------------------------------ MMA issuer
+    for (int kb = 0; kb < args.kb_total; ++kb) {
       const int s = kb % STAGES;
       const uint32_t round = kb / STAGES;
       if (!ptx::mbar_wait(&full[s], round & 1, args.err, kErrTimeoutMma, abort_flag)) break;
@@ -103,8 +130,10 @@ kv_gemm_kernel(const __grid_constant__ CUtensorMap map_y, const __grid_constant_
       const uint32_t b = a + A_BYTES;
 #pragma unroll
       for (int kk = 0; kk < BK / 16; ++kk) {
-        const uint64_t da = ptx::smem_desc_sw128(a + kk * 32, 16, 1024);
-        const uint64_t db = ptx::smem_desc_sw128(b + kk * 16 * 128, B_BOX_BYTES, 1024);
+        const uint64_t da = A_MN ? ptx::smem_desc_sw128(a + kk * 2048, 8192, 1024)
+                                 : ptx::smem_desc_sw128(a + kk * 32, 16, 1024);
+        const uint64_t db = B_MN ? ptx::smem_desc_sw128(b + kk * 2048, 8192, 1024)
+                                 : ptx::smem_desc_sw128(b + kk * 32, 16, 1024);
         ptx::mma_ss(tmem, da, db, IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
       }
       ptx::mma_commit(&empty[s]);
@@ -113,14 +142,15 @@ kv_gemm_kernel(const __grid_constant__ CUtensorMap map_y, const __grid_constant_
   }
   __syncwarp();
 
-  // epilogue: every warp reads its 32-lane quarter of the accumulator.  The
-  // MMA thread always commits acc_full (also after an abort), so this wait
-  // also drains the MMAs before the TMEM is released.
+  // ------------------------------------------------------------------ epilogue
+  // Every warp reads its 32-lane quarter of the accumulator.  The MMA thread
+  // always commits acc_full (also after an abort), so this wait also drains
+  // the MMAs before the TMEM is released.
   const bool ok = ptx::mbar_wait(acc_full, 0, args.err, kErrTimeoutEpilogue, nullptr);
   ptx::tc_fence_after();
   if (ok && !*abort_flag) {
     const int row = m0 + warp * 32 + lane;
-    __nv_bfloat16* out = is_v ? args.out_v : args.out_k;
+    __nv_bfloat16* out = z ? args.out[1] : args.out[0];
 #pragma unroll 1
     for (int c = 0; c < BN / 32; ++c) {
       uint32_t r[32];
@@ -145,6 +175,57 @@ kv_gemm_kernel(const __grid_constant__ CUtensorMap map_y, const __grid_constant_
   if (warp == 2) ptx::tmem_dealloc(tmem, BN);
 }
 
+// Tensor map of a row-major bf16 matrix [rows][cols] (cols contiguous) read in
+// boxes of box_cols x box_rows.
+bool map_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_cols,
+            uint32_t box_rows) {
+  const uint64_t dims[2] = {cols, rows};
+  const uint64_t strides[1] = {cols * 2};
+  const uint32_t box[2] = {box_cols, box_rows};
+  return encode_tensor_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box,
+                           CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// Operand descriptions: base pointer and the row-major shape it is stored in.
+struct Operand {
+  const void* base;
+  uint64_t rows, cols;
+};
+
+// A: K-major = stored [M][K]; M-major = stored [K][M].  B: K-major = stored
+// [N][K]; N-major = stored [K][N].
+template <bool A_MN, bool B_MN>
+cudaError_t launch_gemm(const Operand* a, const Operand* b, __nv_bfloat16* out0,
+                        __nv_bfloat16* out1, int M, int N, int kb_seg0, int kb_total, int batched,
+                        cudaStream_t s) {
+  CUtensorMap ma[2], mb[2];
+  for (int i = 0; i < 2; ++i) {
+    const bool okA = A_MN ? map_2d(&ma[i], a[i].base, a[i].rows, a[i].cols, 64, 64)
+                          : map_2d(&ma[i], a[i].base, a[i].rows, a[i].cols, 64, 128);
+    const bool okB = B_MN ? map_2d(&mb[i], b[i].base, b[i].rows, b[i].cols, 64, 64)
+                          : map_2d(&mb[i], b[i].base, b[i].rows, b[i].cols, 64, 256);
+    if (!okA || !okB) return cudaErrorInvalidValue;
+  }
+  cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<A_MN, B_MN>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  GemmArgs g;
+  g.out[0] = out0;
+  g.out[1] = out1;
+  g.err = device_error_word();
+  g.M = M;
+  g.N = N;
+  g.kb_seg0 = kb_seg0;
+  g.kb_total = kb_total;
+  g.batched = batched;
+  if (!g.err) return cudaErrorInvalidValue;
+  const long long tiles = (long long)(N / BN) * ((M + BM - 1) / BM) * (batched ? 2 : 1);
+  if (tiles > 0x7fffffffll) return cudaErrorInvalidConfiguration;
+  const dim3 grid((unsigned)tiles);
+  gemm_tc_kernel<A_MN, B_MN><<<grid, 128, SMEM_BYTES, s>>>(ma[0], mb[0], ma[1], mb[1], g);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 bool tc_gemm_supported(int M, int K, int N) {
@@ -153,34 +234,39 @@ bool tc_gemm_supported(int M, int K, int N) {
 
 cudaError_t launch_kv_gemm_tc(const void* y, const void* w_k, const void* w_v, void* k, void* v,
                               int M, int K, int N, cudaStream_t s) {
-  CUtensorMap my, mk, mv;
+  // K = y W_k, V = y W_v: A = y [M][K] (K-major), B = W [K][N] (N-major), two problems
+  const Operand a[2] = {{y, (uint64_t)M, (uint64_t)K}, {y, (uint64_t)M, (uint64_t)K}};
+  const Operand b[2] = {{w_k, (uint64_t)K, (uint64_t)N}, {w_v, (uint64_t)K, (uint64_t)N}};
+  return launch_gemm<false, true>(a, b, reinterpret_cast<__nv_bfloat16*>(k),
+                                  reinterpret_cast<__nv_bfloat16*>(v), M, N, K / BK, K / BK, 1, s);
+}
+
+bool tc_gemm_bwd_supported(int S, int E, int N) {
+  // S = B*S_KV rows of y (any count: the last K step of dW reads zeros past
+  // row S-1 from both operands), E = d_embed, N = H_kv*d
+  return S >= 1 && E % BN == 0 && N % BN == 0;
+}
+
+cudaError_t launch_kv_gemm_bwd_tc(const void* y, const void* w_k, const void* w_v,
+                                  const void* dk, const void* dv, void* dy, void* dw_k, void* dw_v,
+                                  int S, int E, int N, cudaStream_t s) {
+  // dW_z = y^T dZ: M = E, N = N, K = S; A = y stored [S][E] (M-major),
+  // B = dZ stored [S][N] (N-major); two problems (dW_k, dW_v)
   {
-    const uint64_t dims[2] = {(uint64_t)K, (uint64_t)M};
-    const uint64_t strides[1] = {(uint64_t)K * 2};
-    const uint32_t box[2] = {BK, BM};
-    if (!encode_tensor_map(&my, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, y, dims, strides, box,
-                           CU_TENSOR_MAP_SWIZZLE_128B))
-      return cudaErrorInvalidValue;
+    const Operand a[2] = {{y, (uint64_t)S, (uint64_t)E}, {y, (uint64_t)S, (uint64_t)E}};
+    const Operand b[2] = {{dk, (uint64_t)S, (uint64_t)N}, {dv, (uint64_t)S, (uint64_t)N}};
+    const int kb = (S + BK - 1) / BK;
+    cudaError_t e = launch_gemm<true, true>(a, b, reinterpret_cast<__nv_bfloat16*>(dw_k),
+                                            reinterpret_cast<__nv_bfloat16*>(dw_v), E, N, kb, kb,
+                                            1, s);
+    if (e != cudaSuccess) return e;
   }
-  {
-    const uint64_t dims[2] = {(uint64_t)N, (uint64_t)K};
-    const uint64_t strides[1] = {(uint64_t)N * 2};
-    const uint32_t box[2] = {64, BK};
-    if (!encode_tensor_map(&mk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w_k, dims, strides, box,
-                           CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_tensor_map(&mv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, w_v, dims, strides, box,
-                           CU_TENSOR_MAP_SWIZZLE_128B))
-      return cudaErrorInvalidValue;
-  }
-  cudaError_t e = cudaFuncSetAttribute(kv_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       SMEM_BYTES);
-  if (e != cudaSuccess) return e;
-  GemmArgs args{reinterpret_cast<__nv_bfloat16*>(k), reinterpret_cast<__nv_bfloat16*>(v),
-                device_error_word(), M, K, N};
-  if (!args.err) return cudaErrorInvalidValue;
-  dim3 grid(2 * (N / BN), (M + BM - 1) / BM);
-  kv_gemm_kernel<<<grid, 128, SMEM_BYTES, s>>>(my, mk, mv, args);
-  return cudaGetLastError();
+  // dy = dK W_k^T + dV W_v^T: M = S, N = E, K = N per segment; A = dZ stored
+  // [S][N] (K-major), B = W_z stored [E][N] (K-major)
+  const Operand a[2] = {{dk, (uint64_t)S, (uint64_t)N}, {dv, (uint64_t)S, (uint64_t)N}};
+  const Operand b[2] = {{w_k, (uint64_t)E, (uint64_t)N}, {w_v, (uint64_t)E, (uint64_t)N}};
+  return launch_gemm<false, false>(a, b, reinterpret_cast<__nv_bfloat16*>(dy), nullptr, S, E,
+                                   N / BK, 2 * (N / BK), 0, s);
 }
 
 }  // namespace lvx

@@ -240,45 +240,55 @@ bwd_simt_kernel(Problem p, const T* __restrict__ q, const T* __restrict__ k,
 
 // ---------------------------------------------------------------- GEMM (K/V recompute fallback)
 
+// C[m][n] = sum over the segments g of sum_k A_g[m][k] B_g[k][n], with A_g and
+// B_g addressed through element strides so that transposed operands need no
+// copy.  64x64 output tile per block, 4x4 per thread, fp32 accumulation.
 template <typename T>
 __global__ void __launch_bounds__(256)
-gemm_simt_kernel(const T* __restrict__ A, const T* __restrict__ Bm, T* __restrict__ C,
-                 int M, int K, int N) {
+gemm_simt_kernel(SimtGemm g) {
   __shared__ float As[16][64 + 1];
   __shared__ float Bs[16][64];
   const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-  const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
+  const int n_tiles = (g.N + 63) / 64;   // tiles run along N first (A-tile reuse in L2)
+  const int m0 = (int)(blockIdx.x / n_tiles) * 64, n0 = (int)(blockIdx.x % n_tiles) * 64;
   float acc[4][4] = {};
-  for (int k0 = 0; k0 < K; k0 += 16) {
-    for (int i = threadIdx.x; i < 64 * 16; i += 256) {
-      const int mm = i / 16, kk = i % 16;
-      const int gm = m0 + mm, gk = k0 + kk;
-      As[kk][mm] = (gm < M && gk < K) ? Elem<T>::to_f(A[(size_t)gm * K + gk]) : 0.f;
-      const int kb = i / 64, nb = i % 64;
-      const int gk2 = k0 + kb, gn = n0 + nb;
-      Bs[kb][nb] = (gk2 < K && gn < N) ? Elem<T>::to_f(Bm[(size_t)gk2 * N + gn]) : 0.f;
+  for (int seg = 0; seg < g.segments; ++seg) {
+    const T* a_ptr = static_cast<const T*>(seg ? g.A[1] : g.A[0]);
+    const T* b_ptr = static_cast<const T*>(seg ? g.B[1] : g.B[0]);
+    for (int k0 = 0; k0 < g.K; k0 += 16) {
+      for (int i = threadIdx.x; i < 64 * 16; i += 256) {
+        const int mm = i / 16, kk = i % 16;
+        const int gm = m0 + mm, gk = k0 + kk;
+        As[kk][mm] = (gm < g.M && gk < g.K)
+                         ? Elem<T>::to_f(a_ptr[(size_t)gm * g.sam + (size_t)gk * g.sak]) : 0.f;
+        const int kb = i / 64, nb = i % 64;
+        const int gk2 = k0 + kb, gn = n0 + nb;
+        Bs[kb][nb] = (gk2 < g.K && gn < g.N)
+                         ? Elem<T>::to_f(b_ptr[(size_t)gk2 * g.sbk + (size_t)gn * g.sbn]) : 0.f;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int kk = 0; kk < 16; ++kk) {
+        float a[4], bb[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) a[i] = As[kk][ty * 4 + i];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) bb[j] = Bs[kk][tx * 4 + j];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], bb[j], acc[i][j]);
+      }
+      __syncthreads();
     }
-    __syncthreads();
-#pragma unroll
-    for (int kk = 0; kk < 16; ++kk) {
-      float a[4], bb[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) a[i] = As[kk][ty * 4 + i];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) bb[j] = Bs[kk][tx * 4 + j];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], bb[j], acc[i][j]);
-    }
-    __syncthreads();
   }
+  T* C = reinterpret_cast<T*>(g.C);
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int gm = m0 + ty * 4 + i, gn = n0 + tx * 4 + j;
-      if (gm < M && gn < N) C[(size_t)gm * N + gn] = Elem<T>::from_f(acc[i][j]);
+      if (gm < g.M && gn < g.N) C[(size_t)gm * g.N + gn] = Elem<T>::from_f(acc[i][j]);
     }
 }
 
@@ -313,14 +323,15 @@ cudaError_t launch_bwd_simt(const Problem& p, lvx_dtype dt, const void* q, const
   return cudaGetLastError();
 }
 
-cudaError_t launch_gemm_simt(const void* y, const void* w, void* out, int M, int K, int N,
-                             lvx_dtype dt, cudaStream_t s) {
-  dim3 grid((N + 63) / 64, (M + 63) / 64);
+cudaError_t launch_gemm_simt(const SimtGemm& g, lvx_dtype dt, cudaStream_t s) {
+  if (g.M < 1 || g.N < 1) return cudaSuccess;
+  const long long tiles = (long long)((g.N + 63) / 64) * ((g.M + 63) / 64);
+  if (tiles > 0x7fffffffll) return cudaErrorInvalidConfiguration;
+  const dim3 grid((unsigned)tiles);
   if (dt == LVX_FP32)
-    gemm_simt_kernel<float><<<grid, 256, 0, s>>>((const float*)y, (const float*)w, (float*)out, M, K, N);
+    gemm_simt_kernel<float><<<grid, 256, 0, s>>>(g);
   else
-    gemm_simt_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
-        (const __nv_bfloat16*)y, (const __nv_bfloat16*)w, (__nv_bfloat16*)out, M, K, N);
+    gemm_simt_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(g);
   return cudaGetLastError();
 }
 

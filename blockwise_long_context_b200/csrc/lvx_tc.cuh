@@ -23,4 +23,11 @@ bool tc_gemm_supported(int M, int K, int N);
 cudaError_t launch_kv_gemm_tc(const void* y, const void* w_k, const void* w_v, void* k, void* v,
                               int M, int K, int N, cudaStream_t s);
 
+// Gradients of the recomputation: dW_k = y^T dK and dW_v = y^T dV in one
+// launch, then dy = dK W_k^T + dV W_v^T.  y [S][E], W [E][N], dK/dV [S][N].
+bool tc_gemm_bwd_supported(int S, int E, int N);
+cudaError_t launch_kv_gemm_bwd_tc(const void* y, const void* w_k, const void* w_v,
+                                  const void* dk, const void* dv, void* dy, void* dw_k, void* dw_v,
+                                  int S, int E, int N, cudaStream_t s);
+
 }  // namespace lvx

@@ -8,7 +8,9 @@ Recipe: ``torch.Generator('cpu').manual_seed(seed)``, ``randn`` in fp32,
 multiplied by the tensor's standard deviation, then rounded to the compute
 dtype (round-to-nearest-even for bf16).  Seeds are
 ``1000 + 10 * config_index + tensor_id`` with tensor ids
-q=0, k=1, v=2, do=3, y=4, w_k=5, w_v=6.
+q=0, k=1, v=2, do=3, y=4, w_k=5, w_v=6, dk=7, dv=8 (dk and dv, unit
+Gaussians, stand in for the gradients the attention backward hands to the
+K/V recomputation when that step is exercised on its own).
 
 The shapes stand in for the LV-XAttn review page's workloads (Llama 3-V,
 long-video cross-attention with S_Q << S_KV, Figure 1 / "The reading"; the
@@ -24,7 +26,7 @@ from typing import Optional
 
 import torch
 
-TENSOR_IDS = {"q": 0, "k": 1, "v": 2, "do": 3, "y": 4, "w_k": 5, "w_v": 6}
+TENSOR_IDS = {"q": 0, "k": 1, "v": 2, "do": 3, "y": 4, "w_k": 5, "w_v": 6, "dk": 7, "dv": 8}
 
 
 @dataclass(frozen=True)
@@ -113,6 +115,8 @@ def make(w: Workload, tensors=("q", "k", "v"), dtype: Optional[torch.dtype] = No
             out[name] = _randn((w.B, w.S_Q, w.H, w.d), seed, w.qkv_std, dt)
         elif name in ("k", "v"):
             out[name] = _randn((w.B, w.S_KV, w.H_kv, w.d), seed, w.qkv_std, dt)
+        elif name in ("dk", "dv"):
+            out[name] = _randn((w.B, w.S_KV, w.H_kv, w.d), seed, 1.0, dt)
         elif name == "do":
             out[name] = _randn((w.B, w.S_Q, w.H, w.d), seed, 1.0, dt)
         elif name == "y":

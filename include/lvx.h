@@ -180,13 +180,37 @@ lvx_status lvx_attn_bwd(const void* q, const void* k, const void* v, const void*
  *   y [B, S_KV, d_embed]; w_k, w_v [d_embed, H_kv*d] row-major; k, v outputs
  *   [B, S_KV, H_kv, d] (= [B, S_KV, H_kv*d]).  fp32 accumulation; bf16 outputs
  *   are rounded to nearest even.
- * Constraints: sizes >= 1, pointers 16-byte aligned.  bf16 requires
- *   d_embed % 64 == 0 and (H_kv*d) % 128 == 0 (tensor-core tiles); otherwise,
- *   and for fp32, a CUDA-core kernel runs.
+ * Constraints: sizes >= 1, pointers 16-byte aligned.  bf16 with
+ *   d_embed % 64 == 0 and (H_kv*d) % 256 == 0 runs on the tensor cores;
+ *   otherwise, and for fp32, a CUDA-core kernel runs.
  */
 lvx_status lvx_kv_recompute(const void* y, const void* w_k, const void* w_v, void* k, void* v,
                             int B, int S_KV, int d_embed, int H_kv, int d, lvx_dtype dt,
                             lvx_stream stream);
+
+/*
+ * Gradients of the key/value recomputation, for training with activation
+ * recomputation (LV-XAttn review page, "What carries the argument" and
+ * Figure 6: the keys and values are regenerated from y in the backward pass,
+ * so the gradient reaching y and the projection weights goes through the
+ * linear map K = y W_k, V = y W_v).  With y, dK, dV flattened to rows
+ * s = b*S_KV + t:
+ *   dW_k = y^T dK,   dW_v = y^T dV              [d_embed, H_kv*d]
+ *   dy   = dK W_k^T + dV W_v^T                  [B, S_KV, d_embed]
+ *   y [B, S_KV, d_embed]; w_k, w_v [d_embed, H_kv*d]; dk, dv [B, S_KV, H_kv, d]
+ *   (the dK, dV of lvx_attn_bwd); outputs dy, dw_k, dw_v are written (not
+ *   accumulated).  All in `dt`; fp32 accumulation, bf16 results rounded to
+ *   nearest even.  Buffers are owned by the caller; inputs and outputs must
+ *   not overlap.
+ * Constraints: sizes >= 1, pointers 16-byte aligned, B*S_KV < 2^31.  bf16 with
+ *   d_embed % 256 == 0 and (H_kv*d) % 256 == 0 runs on the tensor cores (two
+ *   launches); otherwise, and for fp32, CUDA-core kernels run (three
+ *   launches).  Returns LVX_ERR_INVALID_ARG / LVX_ERR_UNSUPPORTED before
+ *   launching anything, LVX_ERR_CUDA if a launch fails.
+ */
+lvx_status lvx_kv_recompute_bwd(const void* y, const void* w_k, const void* w_v, const void* dk,
+                                const void* dv, void* dy, void* dw_k, void* dw_v, int B, int S_KV,
+                                int d_embed, int H_kv, int d, lvx_dtype dt, lvx_stream stream);
 
 /*
  * Synchronises `stream`, then reads and clears the device error word of the

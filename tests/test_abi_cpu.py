@@ -24,7 +24,7 @@ def _declared():
 
 def test_library_exports_every_declared_symbol():
     names = _declared()
-    assert {"lvx_attn_fwd", "lvx_attn_bwd", "lvx_kv_recompute"} <= set(names)
+    assert {"lvx_attn_fwd", "lvx_attn_bwd", "lvx_kv_recompute", "lvx_kv_recompute_bwd"} <= set(names)
     out = subprocess.run(["nm", "-D", "--defined-only", lvx.LIB_PATH], capture_output=True,
                          text=True, check=True).stdout
     exported = set(re.findall(r"\bT (lvx_\w+)", out))
@@ -88,5 +88,18 @@ def test_bwd_and_kv_reject_invalid_arguments():
     assert L.lvx_kv_recompute(P16, P16, None, P16, P16, 1, 4, 64, 1, 64, lvx.LVX_BF16, None) == INVALID
     assert L.lvx_kv_recompute(P16, P16, P16, P16, P16, 1, 0, 64, 1, 64, lvx.LVX_BF16, None) == INVALID
     assert L.lvx_kv_recompute(P16, P16, P16, P16, P16, 1, 4, 64, 1, 64, 9, None) == UNSUPPORTED
+    kvb = [P16] * 8 + [1, 4, 256, 1, 256, lvx.LVX_BF16, None]
+    for i in range(8):   # every pointer is checked
+        bad = list(kvb); bad[i] = None
+        assert L.lvx_kv_recompute_bwd(*bad) == INVALID
+    bad = list(kvb); bad[5] = P16 + 8   # misaligned output
+    assert L.lvx_kv_recompute_bwd(*bad) == INVALID
+    for i in range(8, 13):
+        bad = list(kvb); bad[i] = 0
+        assert L.lvx_kv_recompute_bwd(*bad) == INVALID
+    bad = list(kvb); bad[13] = 9
+    assert L.lvx_kv_recompute_bwd(*bad) == UNSUPPORTED
+    bad = list(kvb); bad[8] = 1 << 16; bad[9] = 1 << 16   # B*S_KV >= 2^31
+    assert L.lvx_kv_recompute_bwd(*bad) == UNSUPPORTED
     assert L.lvx_merge_partials(P16, P16, P16, None, 2, 1, 1, 4, 64, lvx.LVX_BF16, None) == INVALID
     assert L.lvx_merge_partials(P16, P16, P16, P16, 2, 1, 1, 4, 12, lvx.LVX_BF16, None) == UNSUPPORTED
