@@ -17,7 +17,9 @@
 //   dK  += dS^T Q       (SS, dS^T read K-major)  -> TMEM [256+D,256+2D)
 //   dQ_t = dS K         (SS, the same dS^T buffer read MN-major) -> TMEM [128,128+D)
 //   a drain warpgroup reads dQ_t out of TMEM, releases it, and adds it to the
-//   fp32 dQ accumulator with TMA reduce-add (staged in the dS buffer).
+//   fp32 dQ accumulator with TMA reduce-add, staged in the tile's dO slot
+//   (idle once dV has run; the next dO load into that slot waits for the
+//   reduce to have read it), so the reduction overlaps the next tile.
 // dK and dV stay in TMEM for the whole sweep (the group's query heads are
 // summed in place) and are written once at the end.
 #include "lvx_ptx.cuh"
@@ -52,7 +54,15 @@ struct BwdLayout {
   static constexpr uint32_t OFF_DS = OFF_DO + 2 * TILE;    // 128 keys x 128 rows bf16
   static constexpr uint32_t OFF_LSE = OFF_DS + 2 * CHUNK;  // 2 stages x 128 fp32
   static constexpr uint32_t OFF_DD = OFF_LSE + 2 * 512;    // 2 stages x 128 fp32
-  static constexpr uint32_t OFF_BAR = OFF_DD + 2 * 512;
+  // dQ staging, 2 stages x 32 KiB: the dO slots themselves when they are that
+  // large (D = 128), otherwise a buffer of its own
+  static constexpr uint32_t STAGE = 32768;
+  static constexpr bool STAGE_IN_DO = TILE >= STAGE;
+  static constexpr uint32_t OFF_STG = OFF_DD + 2 * 512;
+  static constexpr uint32_t OFF_BAR = OFF_STG + (STAGE_IN_DO ? 0 : 2 * STAGE);
+  __device__ static constexpr uint32_t stage_off(int s) {
+    return STAGE_IN_DO ? OFF_DO + s * TILE : OFF_STG + s * STAGE;
+  }
   static constexpr uint32_t USED = OFF_BAR + 256;
   static constexpr uint32_t SLACK = 768;                   // for aligning the base to 1 KiB
   static constexpr uint32_t BYTES = (USED + SLACK) > 118784 ? (USED + SLACK) : 118784;
@@ -105,7 +115,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
   uint64_t* kv_full = bars + 0;
-  uint64_t* q_full = bars + 1;      // [2]
+  uint64_t* q_full = bars + 1;      // [2] Q, -LSE*log2e, -D of a stage
   uint64_t* q_empty = bars + 3;     // [2]
   uint64_t* s_full = bars + 5;
   uint64_t* dp_full = bars + 6;
@@ -115,8 +125,9 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
   uint64_t* dq_full = bars + 10;
   uint64_t* dq_free = bars + 11;
   uint64_t* mma_drain = bars + 12;
-  uint64_t* stage_free = bars + 13;   // dQ staging (in the dS buffer) read by the TMA
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
+  uint64_t* stage_free = bars + 13;   // [2] a stage's dQ staging read by the TMA
+  uint64_t* do_full = bars + 15;      // [2] dO of a stage
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   if ((uint32_t)(smem - smem_raw) + L::USED > L::BYTES) {   // dynamic smem base not 1 KiB aligned
@@ -139,6 +150,8 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
     for (int s = 0; s < 2; ++s) {
       ptx::mbar_init(&q_full[s], 1);
       ptx::mbar_init(&q_empty[s], 1);
+      ptx::mbar_init(&stage_free[s], 4);
+      ptx::mbar_init(&do_full[s], 1);
     }
     ptx::mbar_init(s_full, 1);
     ptx::mbar_init(dp_full, 1);
@@ -147,7 +160,6 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
     ptx::mbar_init(dq_full, 1);
     ptx::mbar_init(dq_free, 128);
     ptx::mbar_init(mma_drain, 1);
-    ptx::mbar_init(stage_free, 4);
     *abort_flag = 0;
     ptx::fence_barrier_init();
   }
@@ -165,9 +177,8 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
     ptx::setmaxnreg_dec<kRegsControl>();
     if (warp == 0) {
       if (lane == 0) {
-        // ---------------------------------------------------------------- producer
+        // ---------------------------------------------------------------- producer: K, V, Q, LSE, D
         ptx::tma_prefetch_desc(&map_q);
-        ptx::tma_prefetch_desc(&map_do);
         ptx::mbar_arrive_expect_tx(kv_full, 2 * L::TILE);
         for (int c = 0; c < D / 64; ++c) {
           ptx::tma_load_4d(smem + L::OFF_K + c * CHUNK, &map_k, kv_full, 64 * c, g, n0, b);
@@ -179,13 +190,10 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
           const int h = g * grp + i / per_head;
           const int m = m_start + i % per_head;
           if (!ptx::mbar_wait(&q_empty[s], ((i >> 1) & 1) ^ 1, a.err, kErrTimeoutTma, abort_flag)) break;
-          ptx::mbar_arrive_expect_tx(&q_full[s], 2 * L::TILE + 2 * 512);
-          for (int c = 0; c < D / 64; ++c) {
+          ptx::mbar_arrive_expect_tx(&q_full[s], L::TILE + 2 * 512);
+          for (int c = 0; c < D / 64; ++c)
             ptx::tma_load_4d(smem + L::OFF_Q + s * L::TILE + c * CHUNK, &map_q, &q_full[s], 64 * c, h,
                              BROW * m, b);
-            ptx::tma_load_4d(smem + L::OFF_DO + s * L::TILE + c * CHUNK, &map_do, &q_full[s], 64 * c,
-                             h, BROW * m, b);
-          }
           ptx::tma_load_2d(smem + L::OFF_LSE + s * 512, &map_lse, &q_full[s], BROW * m, b * p.H + h);
           ptx::tma_load_2d(smem + L::OFF_DD + s * 512, &map_dd, &q_full[s], BROW * m, b * p.H + h);
           issued = i + 1;
@@ -194,6 +202,30 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
           ptx::mbar_wait(kv_full, 0, a.err, kErrTimeoutTma, nullptr);
           for (int i = issued > 2 ? issued - 2 : 0; i < issued; ++i)
             ptx::mbar_wait(&q_full[i & 1], (i >> 1) & 1, a.err, kErrTimeoutTma, nullptr);
+        }
+      }
+    } else if (warp == 3) {
+      if (lane == 0) {
+        // ---------------------------------------------------------------- producer: dO
+        // dO of tile i goes into slot i&1 once the drain's reduce has read the
+        // dQ of tile i-2 staged there (D = 128) -- that wait is what lets the
+        // reduction run behind the following tile's work
+        ptx::tma_prefetch_desc(&map_do);
+        int issued = 0;
+        for (int i = 0; i < I; ++i) {
+          const int s = i & 1;
+          const int h = g * grp + i / per_head;
+          const int m = m_start + i % per_head;
+          if (!ptx::mbar_wait(&stage_free[s], ((i >> 1) & 1) ^ 1, a.err, kErrTimeoutTma, abort_flag)) break;
+          ptx::mbar_arrive_expect_tx(&do_full[s], L::TILE);
+          for (int c = 0; c < D / 64; ++c)
+            ptx::tma_load_4d(smem + L::OFF_DO + s * L::TILE + c * CHUNK, &map_do, &do_full[s], 64 * c,
+                             h, BROW * m, b);
+          issued = i + 1;
+        }
+        if (*abort_flag) {
+          for (int i = issued > 2 ? issued - 2 : 0; i < issued; ++i)
+            ptx::mbar_wait(&do_full[i & 1], (i >> 1) & 1, a.err, kErrTimeoutTma, nullptr);
         }
       }
     } else if (warp == 1) {
@@ -223,6 +255,9 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
         };
         auto issue_dp_dv = [&](int i) -> bool {
           const uint32_t dos = do_base + (i & 1) * L::TILE;
+          if (!ptx::mbar_wait(&do_full[i & 1], (i >> 1) & 1, a.err, kErrTimeoutMma, abort_flag))
+            return false;
+          ptx::tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {   // dP^T = V dO^T
             const uint32_t off = (kk >> 2) * CHUNK + (kk & 3) * 32;
@@ -266,12 +301,12 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
                         ptx::smem_desc_sw128(qs + kk * 2048, CHUNK, 1024), L::IDESC_DK,
                         (i > 0 || kk > 0) ? 1u : 0u);
           }
+          ptx::mma_commit(&q_empty[s]);   // Q, LSE, D of this stage are no longer read
 #pragma unroll
           for (int kk = 0; kk < BKEY / 16; ++kk)   // dQ_t = dS K
             ptx::mma_ss(tdP, ptx::smem_desc_sw128(ds_base + kk * 2048, CHUNK, 1024),
                         ptx::smem_desc_sw128(k_base + kk * 2048, CHUNK, 1024), L::IDESC_DQ, kk > 0);
           ptx::mma_commit(dq_full);
-          ptx::mma_commit(&q_empty[s]);
           if (i + 1 < I) {
             ok = ptx::mbar_wait(dq_free, i & 1, a.err, kErrTimeoutMma, abort_flag);
             if (!ok) break;
@@ -369,10 +404,6 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
       ptx::tc_fence_before();
       ptx::mbar_arrive(p_ready);
       ok = ptx::mbar_wait(dp_full, i & 1, a.err, kErrTimeoutSoftmax, abort_flag);
-      // the dS buffer doubles as the drain's dQ staging: wait until the TMA has
-      // read the previous tile's pieces
-      if (ok && i > 0)
-        ok = ptx::mbar_wait(stage_free, (i - 1) & 1, a.err, kErrTimeoutSoftmax, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       ptx::tc_fence_after();
@@ -450,13 +481,15 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
     // ------------------------------------------------------------------ dQ drain
     // Warp 12+q reads TMEM lanes 32q..32q+31 (query rows) of dQ_t, releases the
     // columns to the MMA warp, and adds the rows to dQ_acc: 32x32 pieces are
-    // staged 128-byte swizzled in its own 8 KiB of the dS buffer (free between
-    // the dQ MMA and the next tile's dS) and reduced with TMA reduce-add.
+    // staged 128-byte swizzled in its own 8 KiB of the tile's staging slot
+    // (the dO slot for D = 128: its last reader, dV, completed before the dQ
+    // MMA) and reduced with TMA reduce-add; the slot is handed back to the dO
+    // producer once the TMA has read it.
     const int quarter = warp & 3;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    uint8_t* stage = smem + L::OFF_DS + quarter * 8192;
     bool ok = true;
     for (int i = 0; i < I; ++i) {
+      uint8_t* stage = smem + L::stage_off(i & 1) + quarter * 8192;
       const int h = g * grp + i / per_head;
       const int m = m_start + i % per_head;
       const int row0 = BROW * m + quarter * 32;
@@ -497,7 +530,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
       }
       if (lane == 0) {
         bulk_wait_read();
-        ptx::mbar_arrive(stage_free);
+        ptx::mbar_arrive(&stage_free[i & 1]);
       }
       __syncwarp();
     }
