@@ -33,12 +33,12 @@ using namespace ptx;
 constexpr int BKEY = 128;
 constexpr int BROW = 128;
 constexpr int kThreads = 512;
-// Register split (launched at 128 per thread): warpgroup 0 (producer, MMA
-// issuer, allocator) 48, the two elementwise warpgroups 168, the dQ drain
-// warpgroup 128:  128 x 48 + 256 x 168 + 128 x 128 = 65536 = 512 x 128.
-constexpr uint32_t kRegsControl = 48;
+// Register split (launched at 128 per thread): warpgroup 0 (producers, MMA
+// issuer, allocator) 56, the two elementwise warpgroups 168, the dQ drain
+// warpgroup 120:  128 x 56 + 256 x 168 + 128 x 120 = 65536 = 512 x 128.
+constexpr uint32_t kRegsControl = 56;
 constexpr uint32_t kRegsElementwise = 168;
-constexpr uint32_t kRegsDrain = 128;
+constexpr uint32_t kRegsDrain = 120;
 static_assert(128 * kRegsControl + 256 * kRegsElementwise + 128 * kRegsDrain <=
                   65536 / kThreads * kThreads,
               "register split exceeds the launch allocation");
@@ -67,6 +67,7 @@ struct BwdLayout {
   static constexpr uint32_t SLACK = 768;                   // for aligning the base to 1 KiB
   static constexpr uint32_t BYTES = (USED + SLACK) > 118784 ? (USED + SLACK) : 118784;
   static constexpr uint32_t IDESC_SS_KK = ptx::idesc_bf16_f32(128, 128, false, false);
+  static constexpr uint32_t IDESC_DP_HALF = ptx::idesc_bf16_f32(128, 64, false, false);
   static constexpr uint32_t IDESC_DV = ptx::idesc_bf16_f32(128, D, false, true);
   static constexpr uint32_t IDESC_DK = ptx::idesc_bf16_f32(128, D, false, true);
   static constexpr uint32_t IDESC_DQ = ptx::idesc_bf16_f32(128, D, true, true);
@@ -118,16 +119,15 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
   uint64_t* q_full = bars + 1;      // [2] Q, -LSE*log2e, -D of a stage
   uint64_t* q_empty = bars + 3;     // [2]
   uint64_t* s_full = bars + 5;
-  uint64_t* dp_full = bars + 6;
   uint64_t* p_ready = bars + 7;
   uint64_t* ds_ready = bars + 8;
-  // bars[9] unused
   uint64_t* dq_full = bars + 10;
-  uint64_t* dq_free = bars + 11;
   uint64_t* mma_drain = bars + 12;
   uint64_t* stage_free = bars + 13;   // [2] a stage's dQ staging read by the TMA
   uint64_t* do_full = bars + 15;      // [2] dO of a stage
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
+  uint64_t* dp_full = bars + 17;      // [2] dP^T of query rows [64h, 64h+64)
+  uint64_t* dq_free = bars + 19;      // [2] dQ_t columns [64h, 64h+64) read by the drain
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 21);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   if ((uint32_t)(smem - smem_raw) + L::USED > L::BYTES) {   // dynamic smem base not 1 KiB aligned
@@ -154,11 +154,13 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
       ptx::mbar_init(&do_full[s], 1);
     }
     ptx::mbar_init(s_full, 1);
-    ptx::mbar_init(dp_full, 1);
     ptx::mbar_init(p_ready, 256);
     ptx::mbar_init(ds_ready, 256);
     ptx::mbar_init(dq_full, 1);
-    ptx::mbar_init(dq_free, 128);
+    for (int h = 0; h < 2; ++h) {
+      ptx::mbar_init(&dp_full[h], 1);
+      ptx::mbar_init(&dq_free[h], 128);
+    }
     ptx::mbar_init(mma_drain, 1);
     *abort_flag = 0;
     ptx::fence_barrier_init();
@@ -242,7 +244,8 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
         // columns: tcgen05.mma ops of one thread execute in issue order, so the
         // read completes first, and the elementwise warps can start on tile
         // i+1 while the tensor core works on dK_i and dQ_i.  dP_{i+1} reuses the
-        // columns of dQ_i and waits until the drain warps have read them.
+        // columns of dQ_i; it is issued as two 64-query halves, each as soon as
+        // the drain warps have read the 64 dQ columns it overwrites.
         auto issue_s = [&](int i) {
           const uint32_t qs = q_base + (i & 1) * L::TILE;
 #pragma unroll
@@ -259,12 +262,21 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
             return false;
           ptx::tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {   // dP^T = V dO^T
-            const uint32_t off = (kk >> 2) * CHUNK + (kk & 3) * 32;
-            ptx::mma_ss(tdP, ptx::smem_desc_sw128(v_base + off, 16, 1024),
-                        ptx::smem_desc_sw128(dos + off, 16, 1024), L::IDESC_SS_KK, kk > 0);
+          for (int h = 0; h < 2; ++h) {   // dP^T = V dO^T, query rows [64h, 64h+64)
+            if (i > 0) {
+              if (!ptx::mbar_wait(&dq_free[h], (i - 1) & 1, a.err, kErrTimeoutMma, abort_flag))
+                return false;
+              ptx::tc_fence_after();
+            }
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * CHUNK + (kk & 3) * 32;
+              ptx::mma_ss(tdP + 64 * h, ptx::smem_desc_sw128(v_base + off, 16, 1024),
+                          ptx::smem_desc_sw128(dos + off + h * 8192, 16, 1024), L::IDESC_DP_HALF,
+                          kk > 0);
+            }
+            ptx::mma_commit(&dp_full[h]);
           }
-          ptx::mma_commit(dp_full);
           if (!ptx::mbar_wait(p_ready, i & 1, a.err, kErrTimeoutMma, abort_flag)) return false;
           ptx::tc_fence_after();
 #pragma unroll
@@ -307,12 +319,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
             ptx::mma_ss(tdP, ptx::smem_desc_sw128(ds_base + kk * 2048, CHUNK, 1024),
                         ptx::smem_desc_sw128(k_base + kk * 2048, CHUNK, 1024), L::IDESC_DQ, kk > 0);
           ptx::mma_commit(dq_full);
-          if (i + 1 < I) {
-            ok = ptx::mbar_wait(dq_free, i & 1, a.err, kErrTimeoutMma, abort_flag);
-            if (!ok) break;
-            ptx::tc_fence_after();
-            ok = issue_dp_dv(i + 1);
-          }
+          if (i + 1 < I) ok = issue_dp_dv(i + 1);
         }
         ptx::mma_commit(mma_drain);
       }
@@ -403,7 +410,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
       }
       ptx::tc_fence_before();
       ptx::mbar_arrive(p_ready);
-      ok = ptx::mbar_wait(dp_full, i & 1, a.err, kErrTimeoutSoftmax, abort_flag);
+      ok = ptx::mbar_wait(&dp_full[hf], i & 1, a.err, kErrTimeoutSoftmax, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       ptx::tc_fence_after();
@@ -503,10 +510,11 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
         ptx::tmem_ld32(tdP + lane_off + 64 * round, *reinterpret_cast<uint32_t(*)[32]>(&qr[0]));
         ptx::tmem_ld32(tdP + lane_off + 64 * round + 32, *reinterpret_cast<uint32_t(*)[32]>(&qr[32]));
         ptx::tmem_wait_ld();
-        if (round == D / 64 - 1) {
-          ptx::tc_fence_before();
-          ptx::mbar_arrive(dq_free);
-        }
+        // these 64 columns may now take the next tile's dP^T half (with D = 64
+        // the second half of the dP^T columns never held dQ)
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(&dq_free[round]);
+        if (D == 64) ptx::mbar_arrive(&dq_free[1]);
         if (round > 0) {   // the previous round's pieces must have been read by the TMA
           if (lane == 0) bulk_wait_read();
           __syncwarp();
