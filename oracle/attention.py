@@ -10,7 +10,7 @@ Layouts (all numpy arrays, converted to float64 on entry):
   k, v, dk, dv : [B, S_KV, H_kv, d]
   lse          : [B, H, S_Q]   natural-log log-sum-exp of the scaled logits
 
-Readings of the pages that this file fixes (each listed in the design doc):
+Readings of the pages that this file fixes (where the pages are silent or ambiguous):
   * scale s = 1/sqrt(d), d the per-head width, unless given;
   * query head h reads key/value head floor(h / (H / H_kv)) (contiguous
     groups, the repeat-interleave convention for grouped-query attention);
