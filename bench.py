@@ -37,11 +37,12 @@ sys.path.insert(0, ROOT)
 METRIC = "attention fwd+bwd TFLOP/s and % of B200 dense BF16 peak, 1 GPU"
 WORKLOAD = "C2"
 
-# ncu DRAM traffic of the dominant kernel per launch, with the hash of the
-# source file it was taken from (reported only while the source is unchanged).
+# ncu DRAM traffic of the dominant kernel per launch, by (workload, stage), with
+# the hash of the source file it was taken from (reported only for that
+# workload at its full size, and only while the source is unchanged).
 TRAFFIC = {
     # bwd_tc_kernel, one full C2 launch under ncu: 336.65 MB read + 251.77 MB written
-    "bwd": {"bytes": 588.42e6, "source": "blockwise_long_context_b200/csrc/lvx_bwd_tc.cu",
+    ("C2", "bwd"): {"bytes": 588.42e6, "source": "blockwise_long_context_b200/csrc/lvx_bwd_tc.cu",
             "sha": "9f5cd4b801d75107"},
 }
 
@@ -411,7 +412,7 @@ def run_gpu(a):
     dom = max(stages, key=lambda s: stages[s][0])
     t_dom, f_dom, dom_desc = stages[dom]
     achieved = f_dom / (t_dom * 1e-3) / 1e12
-    tr = TRAFFIC.get(dom)
+    tr = None if a.s_kv else TRAFFIC.get((w.name, dom))
     traffic = tr["bytes"] if tr and _file_sha(tr["source"]) == tr["sha"] else None
     # tensor-core dispatch: K/V recompute (1), fwd partials (1) + merge (n_blocks > 1),
     # bwd preprocess + main + dQ finalize (3)
