@@ -129,14 +129,17 @@ def oracle_sample(w, kv_grads: bool = False):
     except Exception:
         cores = os.cpu_count() or 1
     rows = 32
-    sw = w.scaled(S_Q=rows)
+    keys = w.S_KV if w.S_KV <= 262144 else 65536   # cap for the 15M-key shape
+    sw = w.scaled(S_Q=rows, S_KV=keys)
     host = inputs.make(sw, tensors=("q", "k", "v", "do"))
     q, k, v, do = (host[t].double().numpy() for t in ("q", "k", "v", "do"))
     kvw = inputs.make(w, tensors=("w_k", "w_v")) if w.d_embed else None
     t0 = time.perf_counter()
     oracle.attention_fwd(q, k, v, causal=sw.causal)
-    oracle.attention_bwd(q, k, v, do, causal=sw.causal)
-    flops = sw.fwd_flops() + 2.5 * sw.fwd_flops()
+    flops = sw.fwd_flops()
+    if w.backward:
+        oracle.attention_bwd(q, k, v, do, causal=sw.causal)
+        flops += 2.5 * sw.fwd_flops()
     if kvw is not None:
         y = np.random.default_rng(0).standard_normal((rows, w.d_embed))
         oracle.kv_recompute(y, kvw["w_k"].double().numpy(), kvw["w_v"].double().numpy())
@@ -147,8 +150,10 @@ def oracle_sample(w, kv_grads: bool = False):
                                     g[0], g[1])
             flops += 2 * 2 * 2 * rows * w.d_embed * w.H_kv * w.d
     dt = time.perf_counter() - t0
-    desc = (f"fp64 oracle, forward + backward for {rows} of {w.S_Q} query rows over all {w.H} heads "
-            f"and all {w.S_KV} keys, plus K/V recompute of {rows} rows of y"
+    desc = (f"fp64 oracle, forward{' + backward' if w.backward else ''} for {rows} of {w.S_Q} "
+            f"query rows over all {w.H} heads and "
+            f"{'all ' + str(w.S_KV) if keys == w.S_KV else f'the first {keys} of {w.S_KV}'} keys"
+            f"{f', plus K/V recompute of {rows} rows of y' if kvw is not None else ''}"
             f"{' and its gradients' if kv_grads and kvw is not None else ''}; counted FLOPs / time")
     return flops / dt / 1e12, dt, cores, desc
 
@@ -180,11 +185,22 @@ def run_reference(a):
     print(json.dumps(line), flush=True)
 
 
+def _input_bytes(w):
+    """Bytes of the per-step inputs (bf16 / fp32 as the workload computes)."""
+    es = 4 if w.dtype == "f32" else 2
+    qo = w.B * w.S_Q * w.H * w.d * es * (2 if w.backward else 1)
+    if w.d_embed:
+        return qo + (w.B * w.S_KV + 2 * w.H_kv * w.d) * w.d_embed * es
+    return qo + 2 * w.B * w.S_KV * w.H_kv * w.d * es
+
+
 def _config(w, n, kv_grads=False):
     c = {"workload": f"{w.name}: {w.desc}", "B": w.B, "H": w.H, "H_kv": w.H_kv, "d": w.d,
          "S_Q": w.S_Q, "S_KV": w.S_KV, "n_blocks": w.n_blocks, "causal": w.causal,
          "d_embed": w.d_embed, "parallelism": f"replicas{n}" if n > 1 else "single",
-         "l2": "inputs larger than L2: y 512 MiB read and K/V 256 MiB rewritten every step",
+         "l2": (f"inputs larger than L2 (126 MB): {_input_bytes(w) / 2**20:.0f} MiB read every step"
+                + (", K/V 256 MiB rewritten" if w.d_embed else "")) if _input_bytes(w) > 126e6
+               else f"inputs ({_input_bytes(w) / 2**20:.1f} MiB) fit in L2: not a timing workload",
          "flops_counted": "attn fwd 4*B*H*S_Q*S_KV*d + bwd 2.5x fwd + K/V recompute "
                           "2*2*B*S_KV*d_embed*H_kv*d"}
     if kv_grads:
@@ -240,9 +256,16 @@ def run_gpu(a):
 
     recompute = w.d_embed > 0   # K, V regenerated from y every step (else they are inputs)
     kv_grads = recompute and w.backward and a.kv_grads   # + dW_k, dW_v, dy of the recomputation
-    host = inputs.make(w, tensors=("q", "do", "y", "w_k", "w_v") if recompute else ("q", "do", "k", "v"))
-    pinned = {k_: t.pin_memory() for k_, t in host.items()}
-    d = {k_: t.to(dev) for k_, t in pinned.items()}
+    names = (("q", "do") if w.backward else ("q",)) + (("y", "w_k", "w_v") if recompute else ("k", "v"))
+    if _input_bytes(w) > (8 << 30):
+        # tens of GB (the VMME shape): drawn on the device, copied once to pinned host memory
+        d = inputs.make_device(w, tensors=names, device=dev)
+        pinned = {k_: torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t)
+                  for k_, t in d.items()}
+    else:
+        host = inputs.make(w, tensors=names)
+        pinned = {k_: t.pin_memory() for k_, t in host.items()}
+        d = {k_: t.to(dev) for k_, t in pinned.items()}
     B, S_Q, H, hd = d["q"].shape
     if recompute:
         k = torch.empty(w.B, w.S_KV, w.H_kv, w.d, dtype=torch.bfloat16, device=dev)
@@ -251,11 +274,13 @@ def run_gpu(a):
         k, v = d["k"], d["v"]
     out = torch.empty_like(d["q"])
     lse = torch.empty(B, H, S_Q, dtype=torch.float32, device=dev)
-    dq = torch.empty_like(d["q"]); dk = torch.empty_like(k); dv = torch.empty_like(k)
+    dq = dk = dv = None
+    if w.backward:
+        dq = torch.empty_like(d["q"]); dk = torch.empty_like(k); dv = torch.empty_like(k)
     if kv_grads:
         dy = torch.empty_like(d["y"]); dwk = torch.empty_like(d["w_k"]); dwv = torch.empty_like(d["w_v"])
     fws = lvx.fwd_workspace(d["q"], k, w.n_blocks, w.causal)
-    bws = lvx.bwd_workspace(d["q"], k, w.causal)
+    bws = lvx.bwd_workspace(d["q"], k, w.causal) if w.backward else None
     stream = torch.cuda.current_stream()
 
     def step(ev=None):
@@ -326,10 +351,13 @@ def run_gpu(a):
     # End to end through the public API with host buffers.  Every step uploads its
     # inputs from pinned host memory and downloads its gradients; the upload of step
     # i+1 (copy stream) and the download of step i-1 (d2h stream) overlap the compute
-    # of step i, with two device sets of inputs and outputs.  The timed region spans
+    # of step i, with two device sets of inputs and outputs.  When a second set of
+    # inputs would not fit comfortably (the 62.6 GB VMME shape), one set is used and
+    # each upload waits for the previous step's compute.  The timed region spans
     # the first upload through the last download.
     res_names = ("dq", "dk", "dv") if w.backward else ("out",)
     res_dev = {"dq": dq, "dk": dk, "dv": dv, "out": out}
+    res_dev_all = dict(res_dev, lse=lse)
     if kv_grads:   # the gradients reaching y and the weights replace dK, dV as results
         res_names = ("dq", "dy", "dwk", "dwv")
         res_dev.update(dy=dy, dwk=dwk, dwv=dwv)
@@ -338,10 +366,11 @@ def run_gpu(a):
     h2d = sum(t.numel() * t.element_size() for t in pinned.values())
     d2h = sum(t.numel() * t.element_size() for t in res_host.values())
     n_e2e = max(3, min(a.steps, 10))
-    in_sets = [d, {k2: torch.empty_like(t) for k2, t in d.items()}]
-    out_sets = [{"dq": dq, "dk": dk, "dv": dv, "out": out, "lse": lse},
-                {"dq": torch.empty_like(dq), "dk": torch.empty_like(dk), "dv": torch.empty_like(dv),
-                 "out": torch.empty_like(out), "lse": torch.empty_like(lse)}]
+    single = 2 * h2d > 0.4 * torch.cuda.get_device_properties(dev).total_memory
+    in_sets = [d, d] if single else [d, {k2: torch.empty_like(t) for k2, t in d.items()}]
+    res_keys = ("dq", "dk", "dv", "out", "lse") if w.backward else ("out", "lse")
+    out_sets = [{n_: res_dev_all[n_] for n_ in res_keys},
+                {n_: torch.empty_like(res_dev_all[n_]) for n_ in res_keys}]
     if kv_grads:
         out_sets[0].update(dy=dy, dwk=dwk, dwv=dwv)
         out_sets[1].update(dy=torch.empty_like(dy), dwk=torch.empty_like(dwk),
@@ -380,21 +409,25 @@ def run_gpu(a):
     upload(0)
     for i in range(n_e2e):
         cur = i % 2
-        if i + 1 < n_e2e:
+        icur = 0 if single else cur
+        if not single and i + 1 < n_e2e:
             if i >= 1:
                 copy_s.wait_event(in_free[1 - cur])     # step i-1 is done reading that set
             upload(1 - cur)
-        stream.wait_event(in_ready[cur])
+        stream.wait_event(in_ready[icur])
         if i >= 2:
             stream.wait_event(out_free[cur])            # step i-2's download is done
-        run_step(in_sets[cur], out_sets[cur])
-        in_free[cur].record(stream)
+        run_step(in_sets[icur], out_sets[cur])
+        in_free[icur].record(stream)
         out_done[cur].record(stream)
         with torch.cuda.stream(d2h_s):
             d2h_s.wait_event(out_done[cur])
             for name in res_names:
                 res_host[name].copy_(out_sets[cur][name], non_blocking=True)
             out_free[cur].record(d2h_s)
+        if single and i + 1 < n_e2e:
+            copy_s.wait_event(in_free[0])               # step i is done reading the one set
+            upload(0)
     stream.wait_stream(d2h_s)
     stream.wait_stream(copy_s)
     x1.record(stream)
@@ -437,7 +470,8 @@ def run_gpu(a):
                   "frac": merge_gbs / peaks["hbm"], "bytes": merge_bytes},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": n_e2e,
-                "note": "uploads of step i+1 and downloads of step i-1 overlap step i's compute"},
+                "note": ("one input set: each upload follows the previous step's compute" if single
+                         else "uploads of step i+1 and downloads of step i-1 overlap step i's compute")},
         "gpu_launches": launches_per_step * a.steps,
         "clocks": clk,
     }

@@ -12,6 +12,9 @@ q=0, k=1, v=2, do=3, y=4, w_k=5, w_v=6, dk=7, dv=8 (dk and dv, unit
 Gaussians, stand in for the gradients the attention backward hands to the
 K/V recomputation when that step is exercised on its own).
 
+Workloads whose inputs are tens of GB (VMME) are drawn on the device instead
+(``make_device``: same seeds, torch's device generator).
+
 The shapes stand in for the LV-XAttn review page's workloads (Llama 3-V,
 long-video cross-attention with S_Q << S_KV, Figure 1 / "The reading"; the
 pages' Video-MME inputs are not available, synthetic Gaussians replace them)
@@ -89,6 +92,13 @@ WORKLOADS = {
     "C4": Workload("C4", 4, B=2, H=16, H_kv=16, d=128, S_Q=512, S_KV=262144, n_blocks=16,
                    causal=False, dtype="bf16", qkv_std=_R2, backward=True,
                    desc="long-video cross-attention forward + backward, n=16"),
+    # The pages' average Video-MME input for Llama 3-V (LV-XAttn review page, "The reading"):
+    # 5,514 text tokens against 15,279,944 visual tokens; K+V = 62.6 GB in bf16.  Neither
+    # length is a multiple of the 128-row tiles.
+    "VMME": Workload("VMME", 5, B=1, H=32, H_kv=8, d=128, S_Q=5514, S_KV=15279944, n_blocks=8,
+                     causal=False, dtype="bf16", qkv_std=_R2, backward=False,
+                     desc="Video-MME-average-shaped long-video cross-attention forward, "
+                          "Llama-3-V heads"),
 }
 
 
@@ -105,24 +115,51 @@ def _randn(shape, seed: int, std: float, dtype: torch.dtype) -> torch.Tensor:
     return t.to(dtype)
 
 
+def spec(w: Workload, name: str):
+    """(shape, standard deviation) of input tensor ``name`` of workload ``w``."""
+    if name in ("q", "do"):
+        return (w.B, w.S_Q, w.H, w.d), (w.qkv_std if name == "q" else 1.0)
+    if name in ("k", "v"):
+        return (w.B, w.S_KV, w.H_kv, w.d), w.qkv_std
+    if name in ("dk", "dv"):
+        return (w.B, w.S_KV, w.H_kv, w.d), 1.0
+    if name == "y":
+        return (w.B, w.S_KV, w.d_embed), 1.0
+    if name in ("w_k", "w_v"):
+        return (w.d_embed, w.H_kv * w.d), 1.0 / math.sqrt(w.d_embed)
+    raise KeyError(name)
+
+
 def make(w: Workload, tensors=("q", "k", "v"), dtype: Optional[torch.dtype] = None) -> dict:
     """Host tensors for workload ``w`` (contiguous, CPU)."""
     dt = dtype or w.torch_dtype
     out = {}
     for name in tensors:
-        seed = seed_for(w, name)
-        if name == "q":
-            out[name] = _randn((w.B, w.S_Q, w.H, w.d), seed, w.qkv_std, dt)
-        elif name in ("k", "v"):
-            out[name] = _randn((w.B, w.S_KV, w.H_kv, w.d), seed, w.qkv_std, dt)
-        elif name in ("dk", "dv"):
-            out[name] = _randn((w.B, w.S_KV, w.H_kv, w.d), seed, 1.0, dt)
-        elif name == "do":
-            out[name] = _randn((w.B, w.S_Q, w.H, w.d), seed, 1.0, dt)
-        elif name == "y":
-            out[name] = _randn((w.B, w.S_KV, w.d_embed), seed, 1.0, dt)
-        elif name in ("w_k", "w_v"):
-            out[name] = _randn((w.d_embed, w.H_kv * w.d), seed, 1.0 / math.sqrt(w.d_embed), dt)
-        else:
-            raise KeyError(name)
+        shape, std = spec(w, name)
+        out[name] = _randn(shape, seed_for(w, name), std, dt)
+    return out
+
+
+def make_device(w: Workload, tensors=("q", "k", "v"), device="cuda",
+                dtype: Optional[torch.dtype] = None, chunk: int = 1 << 28) -> dict:
+    """Device tensors for workloads too large to draw on the host in reasonable
+    time (the VMME shape: 31 GB per K or V).  Same seeds and distributions as
+    ``make``, drawn with torch's device generator in row-major chunks of
+    ``chunk`` elements; the values are a different stream from ``make``'s, so
+    whatever checks them (the oracle) reads them back from the device."""
+    dt = dtype or w.torch_dtype
+    out = {}
+    for name in tensors:
+        shape, std = spec(w, name)
+        g = torch.Generator(device=device)
+        g.manual_seed(seed_for(w, name))
+        t = torch.empty(shape, dtype=dt, device=device)
+        flat = t.view(-1)
+        for s0 in range(0, flat.numel(), chunk):
+            n = min(chunk, flat.numel() - s0)
+            x = torch.randn(n, generator=g, device=device, dtype=torch.float32)
+            if std != 1.0:
+                x.mul_(std)
+            flat[s0:s0 + n].copy_(x)
+        out[name] = t
     return out
