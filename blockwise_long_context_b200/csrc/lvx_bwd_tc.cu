@@ -21,7 +21,10 @@
 //   (idle once dV has run; the next dO load into that slot waits for the
 //   reduce to have read it), so the reduction overlaps the next tile.
 // dK and dV stay in TMEM for the whole sweep (the group's query heads are
-// summed in place) and are written once at the end.
+// summed in place) and are written once at the end: staged as bf16 in the K
+// and V tiles' shared memory (free once the last dQ MMA completed) in the
+// swizzled layout of a TMA box, then stored with TMA, so the global writes are
+// whole 128-byte rows instead of one key row per lane.
 #include "lvx_ptx.cuh"
 #include "lvx_tc.cuh"
 
@@ -102,6 +105,19 @@ __device__ __forceinline__ void bulk_wait_read() {
 __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
+// Stores a shared-memory tile through a tensor map (TMA, asynchronous).
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, const void* ssrc, int c0,
+                                             int c1, int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(ptx::smem_u32(ssrc)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+// Barrier among the 256 threads of the two elementwise warpgroups.
+__device__ __forceinline__ void elementwise_bar() {
+  asm volatile("bar.sync 1, 256;" ::: "memory");
+}
 
 
 template <int D>
@@ -109,7 +125,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
               const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_do,
               const __grid_constant__ CUtensorMap map_lse, const __grid_constant__ CUtensorMap map_dd,
-              const __grid_constant__ CUtensorMap map_dq, const BwdArgs a) {
+              const __grid_constant__ CUtensorMap map_dq, const __grid_constant__ CUtensorMap map_dk,
+              const __grid_constant__ CUtensorMap map_dv, const BwdArgs a) {
   using L = BwdLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -181,10 +198,12 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
       if (lane == 0) {
         // ---------------------------------------------------------------- producer: K, V, Q, LSE, D
         ptx::tma_prefetch_desc(&map_q);
-        ptx::mbar_arrive_expect_tx(kv_full, 2 * L::TILE);
-        for (int c = 0; c < D / 64; ++c) {
-          ptx::tma_load_4d(smem + L::OFF_K + c * CHUNK, &map_k, kv_full, 64 * c, g, n0, b);
-          ptx::tma_load_4d(smem + L::OFF_V + c * CHUNK, &map_v, kv_full, 64 * c, g, n0, b);
+        if (I > 0) {   // (with no query tile the K and V tiles hold the zero dK, dV instead)
+          ptx::mbar_arrive_expect_tx(kv_full, 2 * L::TILE);
+          for (int c = 0; c < D / 64; ++c) {
+            ptx::tma_load_4d(smem + L::OFF_K + c * CHUNK, &map_k, kv_full, 64 * c, g, n0, b);
+            ptx::tma_load_4d(smem + L::OFF_V + c * CHUNK, &map_v, kv_full, 64 * c, g, n0, b);
+          }
         }
         int issued = 0;
         for (int i = 0; i < I; ++i) {
@@ -200,7 +219,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
           ptx::tma_load_2d(smem + L::OFF_DD + s * 512, &map_dd, &q_full[s], BROW * m, b * p.H + h);
           issued = i + 1;
         }
-        if (*abort_flag) {
+        if (*abort_flag && I > 0) {
           ptx::mbar_wait(kv_full, 0, a.err, kErrTimeoutTma, nullptr);
           for (int i = issued > 2 ? issued - 2 : 0; i < issued; ++i)
             ptx::mbar_wait(&q_full[i & 1], (i >> 1) & 1, a.err, kErrTimeoutTma, nullptr);
@@ -451,14 +470,17 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
       ok = __all_sync(0xffffffffu, ok && !*abort_flag);
       ptx::tc_fence_after();
     }
-    const bool write = key < p.S_KV;
-    const size_t off = (((size_t)b * p.S_KV + key) * p.H_kv + g) * D;
+    // Stage: dV into the V tile, dK (times the softmax scale) into the K tile.
+    // Thread (hf, key j) owns head-width columns [hf D/2, hf D/2 + D/2) of row
+    // j: 16-byte units of the 128-byte row of chunk col/64, at the swizzled
+    // position the TMA box layout gives them.  Every elementwise thread passes
+    // the barrier below, whatever its ok flag, so none can be stranded.
     constexpr int HALF = D / 2;
 #pragma unroll 1
     for (int which = 0; which < 2; ++which) {
       const uint32_t tacc = (which == 0 ? tdV : tdK) + lane_off + HALF * hf;
       const float mul = which == 0 ? 1.f : p.scale;
-      __nv_bfloat16* out = (which == 0 ? a.dv : a.dk) + off + HALF * hf;
+      uint8_t* stg = smem + (which == 0 ? L::OFF_V : L::OFF_K) + j * 128;
 #pragma unroll 1
       for (int c = 0; c < HALF / 32; ++c) {
         uint32_t r[32];
@@ -469,19 +491,28 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
 #pragma unroll
           for (int e = 0; e < 32; ++e) r[e] = 0u;
         }
-        if (write && ok) {
-          uint4* dst = reinterpret_cast<uint4*>(out + 32 * c);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint4 u;
-            u.x = ptx::pack_bf16x2(__uint_as_float(r[8 * q + 0]) * mul, __uint_as_float(r[8 * q + 1]) * mul);
-            u.y = ptx::pack_bf16x2(__uint_as_float(r[8 * q + 2]) * mul, __uint_as_float(r[8 * q + 3]) * mul);
-            u.z = ptx::pack_bf16x2(__uint_as_float(r[8 * q + 4]) * mul, __uint_as_float(r[8 * q + 5]) * mul);
-            u.w = ptx::pack_bf16x2(__uint_as_float(r[8 * q + 6]) * mul, __uint_as_float(r[8 * q + 7]) * mul);
-            dst[q] = u;
-          }
+        for (int q = 0; q < 4; ++q) {
+          const int col = HALF * hf + 32 * c + 8 * q;
+          uint4 u;
+          u.x = ptx::pack_bf16x2(__uint_as_float(r[8 * q + 0]) * mul, __uint_as_float(r[8 * q + 1]) * mul);
+          u.y = ptx::pack_bf16x2(__uint_as_float(r[8 * q + 2]) * mul, __uint_as_float(r[8 * q + 3]) * mul);
+          u.z = ptx::pack_bf16x2(__uint_as_float(r[8 * q + 4]) * mul, __uint_as_float(r[8 * q + 5]) * mul);
+          u.w = ptx::pack_bf16x2(__uint_as_float(r[8 * q + 6]) * mul, __uint_as_float(r[8 * q + 7]) * mul);
+          *reinterpret_cast<uint4*>(stg + (col >> 6) * CHUNK + ((((col & 63) >> 3) ^ (j & 7)) << 4)) = u;
         }
       }
+    }
+    ptx::fence_proxy_async_smem();
+    elementwise_bar();
+    // One thread stores both tiles (rows past S_KV are clipped by the TMA unit).
+    if (warp == 4 && lane == 0 && ok && !*abort_flag) {
+      for (int c = 0; c < D / 64; ++c) {
+        tma_store_4d(&map_dv, smem + L::OFF_V + c * CHUNK, 64 * c, g, n0, b);
+        tma_store_4d(&map_dk, smem + L::OFF_K + c * CHUNK, 64 * c, g, n0, b);
+      }
+      bulk_commit();
+      bulk_wait_all();
     }
   } else {
     ptx::setmaxnreg_dec<kRegsDrain>();
@@ -561,7 +592,7 @@ cudaError_t launch(const Problem& p, const void* q, const void* k, const void* v
                    const void* dout, const float* lse, const float* Dv, float* dq_acc, void* dk,
                    void* dv, cudaStream_t s) {
   using L = BwdLayout<D>;
-  CUtensorMap mq, mk, mv, mdo, mlse, mdd, mdq;
+  CUtensorMap mq, mk, mv, mdo, mlse, mdd, mdq, mdk, mdv;
   {
     const uint64_t dims[4] = {(uint64_t)D, (uint64_t)p.H, (uint64_t)p.S_Q, (uint64_t)p.B};
     const uint64_t str[3] = {(uint64_t)D * 4, (uint64_t)p.H * D * 4, (uint64_t)p.S_Q * p.H * D * 4};
@@ -587,6 +618,10 @@ cudaError_t launch(const Problem& p, const void* q, const void* k, const void* v
     if (!encode_tensor_map(&mk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, k, dims, str, box,
                            CU_TENSOR_MAP_SWIZZLE_128B) ||
         !encode_tensor_map(&mv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, v, dims, str, box,
+                           CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_tensor_map(&mdk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, dk, dims, str, box,
+                           CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_tensor_map(&mdv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, dv, dims, str, box,
                            CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
   }
@@ -615,7 +650,7 @@ cudaError_t launch(const Problem& p, const void* q, const void* k, const void* v
   cudaError_t e = cudaFuncSetAttribute(bwd_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        L::BYTES);
   if (e != cudaSuccess) return e;
-  bwd_tc_kernel<D><<<(unsigned)grid, kThreads, L::BYTES, s>>>(mq, mk, mv, mdo, mlse, mdd, mdq, a);
+  bwd_tc_kernel<D><<<(unsigned)grid, kThreads, L::BYTES, s>>>(mq, mk, mv, mdo, mlse, mdd, mdq, mdk, mdv, a);
   return cudaGetLastError();
 }
 
