@@ -202,7 +202,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
           const uint32_t v_base = ptx::smem_u32(smem + L::OFF_V);
           auto issue_s = [&](int t, int j) {
             const int s = j % K_STAGES;
-  #pragma unroll
+#pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               const uint32_t off = (kk >> 2) * CHUNK + (kk & 3) * 32;
               const uint64_t da = ptx::smem_desc_sw128(q_base + t * L::TILE + off, 16, 1024);
@@ -213,7 +213,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
           };
           auto issue_pv = [&](int t, int j) {
             const int s = j % V_STAGES;
-  #pragma unroll
+#pragma unroll
             for (int kk = 0; kk < BKV / 16; ++kk) {
               const uint64_t db =
                   ptx::smem_desc_sw128(v_base + s * L::TILE + kk * 16 * 128, CHUNK, 1024);
@@ -282,72 +282,27 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
       ptx::tmem_wait_ld();
       const int key0 = kb0 + BKV * j;
       const bool need_mask = (key0 + BKV > kb1) || (p.causal && key0 + BKV - 1 > row0_tile);
-      if (need_mask) {
-        const int lim = p.causal ? min(kb1, row + 1) : kb1;   // keys [key0, lim) visible
-#pragma unroll
-        for (int i = 0; i < 128; ++i)
-          if (key0 + i >= lim) sr[i] = __float_as_uint(-INFINITY);
-      }
-      // row max: four independent chains of 3-input maxima (a single chain is
-      // latency-bound), then combined
-      float m4[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) m4[q] = fmaxf(__uint_as_float(sr[32 * q]), __uint_as_float(sr[32 * q + 1]));
-#pragma unroll
-      for (int i = 2; i < 32; i += 2)
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          m4[q] = fmax3(m4[q], __uint_as_float(sr[32 * q + i]), __uint_as_float(sr[32 * q + i + 1]));
-      const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-      const float m_tile = mx * sl2;
-      const bool resc = m_tile > m_ref + kRescaleThreshold;
-      float alpha = 1.f;
-      if (resc) {
-        alpha = ex2(m_ref - m_tile);   // 0 when m_ref is -inf
-        m_ref = m_tile;
-        l_sum *= alpha;
-      }
-      if (j > 0 && __any_sync(0xffffffffu, resc)) {
-        // O_t is quiescent here: P_t V of tile j-1 finished before S_t of tile j was issued
-#pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          ptx::tmem_ld32(tO + c * 32, o);
-          ptx::tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          ptx::tmem_st32(tO + c * 32, o);
-        }
-      }
-      const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
-      if (need_mask) {
-        // masked tiles: every exponential on the special-function unit (exact 0 for -inf)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float p0 = ex2(fmaf(__uint_as_float(sr[32 * c + 2 * i]), sl2, -m_use));
-            const float p1 = ex2(fmaf(__uint_as_float(sr[32 * c + 2 * i + 1]), sl2, -m_use));
-            l_sum += p0 + p1;
-            pk[i] = ptx::pack_bf16x2(p0, p1);
-          }
-          ptx::tmem_st16(tS + 16 * c, pk);
-        }
-      } else {
-        // packed pairs: x = s*scale - m with FFMA2, one pair in kPolyEvery through the
-        // FMA-pipe polynomial and the rest on the SFU, row sum with FADD2
+      // Steady state (an unmasked tile once the row has a running maximum): P is
+      // computed with the running maximum straight away, and the tile's maximum
+      // is found in the same pass instead of before it.  Only if it exceeds the
+      // running maximum by more than the threshold (for any row of the warp) is
+      // that P discarded -- nothing has been released yet -- and the tile redone
+      // below with the maximum moved, exactly as a first tile is.
+      bool done = false;
+      if (!need_mask && m_ref != -INFINITY) {
         const uint64_t sl2x2 = pk2(sl2, sl2);
-        const uint64_t negm2 = pk2(-m_use, -m_use);
-        uint64_t acc2 = pk2(0.f, 0.f);
+        const uint64_t negm2 = pk2(-m_ref, -m_ref);
+        uint64_t acc2 = pk2(0.f, 0.f), acc2b = pk2(0.f, 0.f);
+        float mc[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const uint64_t s2 = pk2(__uint_as_float(sr[32 * c + 2 * i]),
-                                    __uint_as_float(sr[32 * c + 2 * i + 1]));
-            const uint64_t x2 = ffma2(s2, sl2x2, negm2);
+            const float s0 = __uint_as_float(sr[32 * c + 2 * i]);
+            const float s1 = __uint_as_float(sr[32 * c + 2 * i + 1]);
+            mc[i & 3] = fmax3(mc[i & 3], s0, s1);
+            const uint64_t x2 = ffma2(pk2(s0, s1), sl2x2, negm2);
             uint64_t e2;
             if (i % kPolyEvery == kPolyEvery - 1) {
               e2 = exp2_poly2(x2);
@@ -356,16 +311,107 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
               upk2(x2, x0, x1);
               e2 = pk2(ex2(x0), ex2(x1));
             }
-            acc2 = fadd2(acc2, e2);
+            if (i & 1) acc2b = fadd2(acc2b, e2); else acc2 = fadd2(acc2, e2);
             float p0, p1;
             upk2(e2, p0, p1);
             pk[i] = ptx::pack_bf16x2(p0, p1);
           }
           ptx::tmem_st16(tS + 16 * c, pk);
         }
-        float a0, a1;
-        upk2(acc2, a0, a1);
-        l_sum += a0 + a1;
+        const float m_tile = fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3])) * sl2;
+        if (!__any_sync(0xffffffffu, m_tile > m_ref + kRescaleThreshold)) {
+          float a0, a1;
+          upk2(fadd2(acc2, acc2b), a0, a1);
+          l_sum += a0 + a1;
+          done = true;
+        }
+      }
+      if (!done) {
+        if (need_mask) {
+          const int lim = p.causal ? min(kb1, row + 1) : kb1;   // keys [key0, lim) visible
+#pragma unroll
+          for (int i = 0; i < 128; ++i)
+            if (key0 + i >= lim) sr[i] = __float_as_uint(-INFINITY);
+        }
+        // row max: four independent chains of 3-input maxima (a single chain is
+        // latency-bound), then combined
+        float m4[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) m4[q] = fmaxf(__uint_as_float(sr[32 * q]), __uint_as_float(sr[32 * q + 1]));
+#pragma unroll
+        for (int i = 2; i < 32; i += 2)
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            m4[q] = fmax3(m4[q], __uint_as_float(sr[32 * q + i]), __uint_as_float(sr[32 * q + i + 1]));
+        const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+        const float m_tile = mx * sl2;
+        const bool resc = m_tile > m_ref + kRescaleThreshold;
+        float alpha = 1.f;
+        if (resc) {
+          alpha = ex2(m_ref - m_tile);   // 0 when m_ref is -inf
+          m_ref = m_tile;
+          l_sum *= alpha;
+        }
+        if (j > 0 && __any_sync(0xffffffffu, resc)) {
+          // O_t is quiescent here: P_t V of tile j-1 finished before S_t of tile j was issued
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            ptx::tmem_ld32(tO + c * 32, o);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            ptx::tmem_st32(tO + c * 32, o);
+          }
+        }
+        const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
+        if (need_mask) {
+          // masked tiles: every exponential on the special-function unit (exact 0 for -inf)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float p0 = ex2(fmaf(__uint_as_float(sr[32 * c + 2 * i]), sl2, -m_use));
+              const float p1 = ex2(fmaf(__uint_as_float(sr[32 * c + 2 * i + 1]), sl2, -m_use));
+              l_sum += p0 + p1;
+              pk[i] = ptx::pack_bf16x2(p0, p1);
+            }
+            ptx::tmem_st16(tS + 16 * c, pk);
+          }
+        } else {
+          // packed pairs: x = s*scale - m with FFMA2, one pair in kPolyEvery through the
+          // FMA-pipe polynomial and the rest on the SFU, row sum with FADD2
+          const uint64_t sl2x2 = pk2(sl2, sl2);
+          const uint64_t negm2 = pk2(-m_use, -m_use);
+          uint64_t acc2 = pk2(0.f, 0.f);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const uint64_t s2 = pk2(__uint_as_float(sr[32 * c + 2 * i]),
+                                      __uint_as_float(sr[32 * c + 2 * i + 1]));
+              const uint64_t x2 = ffma2(s2, sl2x2, negm2);
+              uint64_t e2;
+              if (i % kPolyEvery == kPolyEvery - 1) {
+                e2 = exp2_poly2(x2);
+              } else {
+                float x0, x1;
+                upk2(x2, x0, x1);
+                e2 = pk2(ex2(x0), ex2(x1));
+              }
+              acc2 = fadd2(acc2, e2);
+              float p0, p1;
+              upk2(e2, p0, p1);
+              pk[i] = ptx::pack_bf16x2(p0, p1);
+            }
+            ptx::tmem_st16(tS + 16 * c, pk);
+          }
+          float a0, a1;
+          upk2(acc2, a0, a1);
+          l_sum += a0 + a1;
+        }
       }
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
