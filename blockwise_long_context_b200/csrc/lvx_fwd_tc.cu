@@ -62,9 +62,9 @@ struct FwdLayout {
 
 struct FwdArgs {
   Problem p;
-  __nv_bfloat16* out;   // final output (n_blocks == 1)
+  __nv_bfloat16* out;   // final output (when o_parts is null)
   float* lse;
-  float* o_parts;       // partials (n_blocks > 1)
+  float* o_parts;       // block partials (null: write the final output)
   float* l_parts;
   unsigned int* err;
   int n_qp;             // query tile pairs per (batch, head)
@@ -437,7 +437,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
         for (int i = 0; i < 32; ++i) o[i] = 0u;
       }
       if (!write) continue;
-      if (p.n_blocks == 1) {
+      if (a.o_parts == nullptr) {   // the final output (one block), else the block partials
         uint4* dst = reinterpret_cast<uint4*>(
             a.out + (((size_t)b * p.S_Q + row) * p.H + h) * D + c * 32);
 #pragma unroll
@@ -458,7 +458,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
       }
     }
     if (write) {
-      if (p.n_blocks == 1)
+      if (a.o_parts == nullptr)
         a.lse[((size_t)b * p.H + h) * p.S_Q + row] = Lrow;
       else
         a.l_parts[prow] = Lrow;

@@ -117,7 +117,7 @@ fwd_simt_kernel(Problem p, const T* __restrict__ q, const T* __restrict__ k,
   const bool seen = m_run != -INFINITY;
   const float inv_l = seen ? 1.f / l_run : 0.f;
   const float L = seen ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
-  if (p.n_blocks == 1) {
+  if (o_parts == nullptr) {   // the final output (one block), else the block partials
     for (int t = 0; t < 4; ++t) {
       const int c = lane + 32 * t;
       if (c < d) out[(((size_t)b * p.S_Q + r) * p.H + h) * d + c] = Elem<T>::from_f(o[t] * inv_l);

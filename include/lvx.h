@@ -132,6 +132,24 @@ lvx_status lvx_attn_fwd_noalloc(const void* q, const void* k, const void* v, voi
                                 lvx_stream stream);
 
 /*
+ * Block partials without the merge: the per-block step of lvx_attn_fwd on its
+ * own, for callers that merge elsewhere -- in LV-XAttn each worker keeps one
+ * stationary shard of the keys and values and its partials are combined with
+ * the other workers' (LV-XAttn review page, "The reading" and Figure 3 /
+ * Algorithm 1; the rescaling is lvx_merge_partials).
+ *   q [B,S_Q,H,d], k, v [B,S_KV,H_kv,d] (device, dtype dt): the caller's shard
+ *   of the keys and values, cut into n_blocks blocks as lvx_attn_fwd cuts them.
+ *   O_parts [n_blocks, B, H, S_Q, d] float32 and L_parts [n_blocks, B, H, S_Q]
+ *   float32 (device, caller-owned, 16-byte aligned): the normalised partial
+ *   outputs and their natural-log log-sum-exp; an empty block writes (0, -inf).
+ * Non-causal only (a shard of a cross-attention key sequence): the same
+ * constraints and errors as lvx_attn_fwd with causal = 0 and no workspace.
+ */
+lvx_status lvx_attn_fwd_partials(const void* q, const void* k, const void* v, float* O_parts,
+                                 float* L_parts, int B, int H, int H_kv, int S_Q, int S_KV, int d,
+                                 int n_blocks, lvx_dtype dt, float scale, lvx_stream stream);
+
+/*
  * Merge of block partials on its own (the rescaling step of lvx_attn_fwd),
  * for callers that produce the partials elsewhere, e.g. one block per GPU.
  *   O_parts [n, B, H, S_Q, d] float32, L_parts [n, B, H, S_Q] float32 (device)

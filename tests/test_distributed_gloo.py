@@ -1,0 +1,91 @@
+"""LV-XAttn's exchange across ranks, on CPU with the gloo backend.
+
+The distributed forward keeps one key/value shard per rank, gathers every
+rank's block partials (O_i, L_i) and merges them.  These tests check the host
+side of that on CPU: the shard partition, and that the partials of each
+rank's shard, gathered over two and three gloo ranks by ``gather_partials``
+(the function the GPU path uses), merge to exact attention on every rank.
+The partials and the merge here come from the fp64 oracle -- the library's
+kernels need a GPU; ``tests/test_parity_distributed.py`` runs those.
+"""
+
+import os
+import socket
+import sys
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+@pytest.mark.parametrize("S_KV,world", [(1000, 2), (1000, 3), (7, 3), (64, 8), (5, 5)])
+def test_shards_partition_the_keys(S_KV, world):
+    sys.path.insert(0, ROOT)
+    from blockwise_long_context_b200.distributed import shard_bounds
+    bounds = [shard_bounds(S_KV, world, r) for r in range(world)]
+    assert bounds[0][0] == 0 and bounds[-1][1] == S_KV
+    for (lo, hi), (lo2, _) in zip(bounds, bounds[1:]):
+        assert lo <= hi == lo2
+    per = -(-S_KV // world)
+    assert all(hi - lo <= per for lo, hi in bounds)
+
+
+def _to_kernel_layout(O, L):
+    """oracle partials O [n, B, R, H, d], L [n, B, H, R] -> kernel layout
+    O [n, B, H, R, d], L [n, B, H, R] (float32 tensors, as the GPU path gathers)."""
+    return (torch.from_numpy(np.ascontiguousarray(np.transpose(O, (0, 1, 3, 2, 4)))).float(),
+            torch.from_numpy(np.ascontiguousarray(L)).float())
+
+
+def _worker(rank, world, port, n_local, results):
+    import datetime
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    import oracle
+    from blockwise_long_context_b200.distributed import gather_partials, shard_bounds
+    rng = np.random.default_rng(7)                 # the same full problem on every rank
+    B, S_Q, H, H_kv, d, S_KV = 2, 5, 4, 2, 8, 23
+    q = rng.standard_normal((B, S_Q, H, d))
+    k = rng.standard_normal((B, S_KV, H_kv, d))
+    v = rng.standard_normal((B, S_KV, H_kv, d))
+    lo, hi = shard_bounds(S_KV, world, rank)
+    O, L = oracle.block_partials(q, k[:, lo:hi], v[:, lo:hi], n_local)
+    o_loc, l_loc = _to_kernel_layout(O, L)
+    o_all, l_all = gather_partials(o_loc, l_loc)
+    assert o_all.shape[0] == world * n_local and l_all.shape[0] == world * n_local
+    # back to the oracle layout, merged by the oracle
+    O_all = np.transpose(o_all.double().numpy(), (0, 1, 3, 2, 4))
+    out, lse = oracle.merge_partials(O_all, l_all.double().numpy())
+    o_ref, l_ref = oracle.attention_fwd(q, k, v)
+    results[rank] = (float(np.abs(out - o_ref).max()), float(np.abs(lse - l_ref).max()),
+                     o_all.double().numpy().sum())
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,n_local", [(2, 1), (3, 2)])
+def test_gathered_shard_partials_merge_to_attention(world, n_local):
+    port = _free_port()
+    with mp.Manager() as m:
+        results = m.dict()
+        mp.spawn(_worker, args=(world, port, n_local, results), nprocs=world, join=True)
+        res = dict(results)
+    assert sorted(res) == list(range(world))
+    for rank, (eo, el, _) in res.items():
+        # float32 partials (as gathered on GPUs) against the fp64 definition
+        assert eo < 1e-5 and el < 1e-5, (rank, eo, el)
+    # every rank gathered the same tensors
+    sums = {r: v[2] for r, v in res.items()}
+    assert len(set(sums.values())) == 1

@@ -1,0 +1,112 @@
+"""GPU parity of the per-shard partials and of LV-XAttn's sharded forward.
+
+``lvx_attn_fwd_partials`` computes one key/value shard's block partials
+(O_i, L_i) without merging them; ``distributed.xattn_forward_sharded`` runs
+it on every rank, all-gathers the partials and merges them with
+``lvx_merge_partials`` (LV-XAttn review page, "The reading" and Figure 3 /
+Algorithm 1).  Runs here get one GPU, so the several ranks are emulated in
+one process -- each shard's partials computed separately and concatenated in
+rank order, which is what the all-gather produces -- and the real
+torch.distributed path runs with a one-rank NCCL group.  Every result is
+checked against the fp64 oracle's unsplit attention.
+"""
+
+import datetime
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from blockwise_long_context_b200 import binding as lvx
+from blockwise_long_context_b200 import inputs
+from blockwise_long_context_b200.distributed import shard_bounds, xattn_forward_sharded
+from tests._parity import compare
+
+pytestmark = pytest.mark.gpu
+
+
+def _problem(B, H, H_kv, d, S_Q, S_KV, dtype="bf16", seed_cfg=1):
+    base = inputs.WORKLOADS["C0" if dtype == "f32" else "C1"]
+    w = base.scaled(B=B, H=H, H_kv=H_kv, d=d, S_Q=S_Q, S_KV=S_KV, n_blocks=1, causal=False,
+                    dtype=dtype)
+    host = inputs.make(w)
+    return w, host
+
+
+def _oracle(host):
+    q, k, v = (host[t].double().numpy() for t in ("q", "k", "v"))
+    return oracle.attention_fwd(q, k, v)
+
+
+@pytest.mark.parametrize("dtype,d,n", [("bf16", 128, 1), ("bf16", 128, 3), ("bf16", 64, 2),
+                                       ("f32", 64, 2)])
+def test_shard_partials_match_oracle_partials(dtype, d, n):
+    w, host = _problem(2, 4, 2, d, 200, 700, dtype)
+    dev = {t: x.cuda() for t, x in host.items()}
+    O = torch.empty(n, w.B, w.H, w.S_Q, w.d, dtype=torch.float32, device="cuda")
+    L = torch.empty(n, w.B, w.H, w.S_Q, dtype=torch.float32, device="cuda")
+    lvx.lvx_attn_fwd_partials(dev["q"], dev["k"], dev["v"], O, L)
+    lvx.lvx_last_device_error()
+    torch.cuda.synchronize()
+    q, k, v = (host[t].double().numpy() for t in ("q", "k", "v"))
+    O_r, L_r = oracle.block_partials(q, k, v, n)
+    compare(O, np.transpose(O_r, (0, 1, 3, 2, 4)), w.dtype, f"partials {dtype} d={d} n={n}: O")
+    compare(L, L_r, w.dtype, f"partials {dtype} d={d} n={n}: L",
+            rel_rms=1e-4 if dtype == "bf16" else 1e-6)
+
+
+@pytest.mark.parametrize("world,n_local,S_KV", [(2, 1, 1024), (3, 2, 1000), (8, 1, 4099)])
+def test_sharded_forward_emulated_ranks(world, n_local, S_KV):
+    """Each emulated rank computes its shard's partials; concatenated in rank
+    order (the all-gather's layout) and merged they give attention over the
+    whole key/value sequence."""
+    w, host = _problem(1, 8, 2, 128, 300, S_KV)
+    dev = {t: x.cuda() for t, x in host.items()}
+    Os, Ls = [], []
+    for r in range(world):
+        lo, hi = shard_bounds(S_KV, world, r)
+        O = torch.empty(n_local, w.B, w.H, w.S_Q, w.d, dtype=torch.float32, device="cuda")
+        L = torch.empty(n_local, w.B, w.H, w.S_Q, dtype=torch.float32, device="cuda")
+        lvx.lvx_attn_fwd_partials(dev["q"], dev["k"][:, lo:hi].contiguous(),
+                                  dev["v"][:, lo:hi].contiguous(), O, L)
+        Os.append(O); Ls.append(L)
+    out = torch.empty_like(dev["q"])
+    lse = torch.empty(w.B, w.H, w.S_Q, dtype=torch.float32, device="cuda")
+    lvx.lvx_merge_partials(torch.cat(Os), torch.cat(Ls), out, lse)
+    lvx.lvx_last_device_error()
+    torch.cuda.synchronize()
+    o_ref, l_ref = _oracle(host)
+    compare(out, o_ref, "bf16", f"sharded x{world}: O")
+    compare(lse, l_ref, "bf16", f"sharded x{world}: LSE", rel_rms=1e-4)
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def test_sharded_forward_through_torch_distributed():
+    """The real path: NCCL process group (one rank on this GPU), partials,
+    all-gather, merge."""
+    import torch.distributed as dist
+    w, host = _problem(2, 4, 4, 128, 256, 2048)
+    dev = {t: x.cuda() for t, x in host.items()}
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    os.environ["MASTER_PORT"] = str(_free_port())
+    dist.init_process_group("nccl", rank=0, world_size=1, timeout=datetime.timedelta(seconds=60),
+                            device_id=torch.device("cuda", 0))
+    try:
+        lo, hi = shard_bounds(w.S_KV, 1, 0)
+        out, lse = xattn_forward_sharded(dev["q"], dev["k"][:, lo:hi], dev["v"][:, lo:hi],
+                                         n_local_blocks=4)
+        lvx.lvx_last_device_error()
+        torch.cuda.synchronize()
+    finally:
+        dist.destroy_process_group()
+    o_ref, l_ref = _oracle(host)
+    compare(out, o_ref, "bf16", "torch.distributed: O")
+    compare(lse, l_ref, "bf16", "torch.distributed: LSE", rel_rms=1e-4)
