@@ -90,36 +90,6 @@ struct BwdArgs {
   int n_items;  // key tiles over all (batch, kv head)
 };
 
-// Adds a shared-memory tile into global memory through a tensor map (TMA
-// reduce-add in L2, asynchronous; the tile may be reused after bulk_wait_read).
-__device__ __forceinline__ void tma_reduce_add_4d(const CUtensorMap* map, const void* ssrc, int c0,
-                                                  int c1, int c2, int c3) {
-  asm volatile(
-      "cp.reduce.async.bulk.tensor.4d.global.shared::cta.add.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
-          reinterpret_cast<uint64_t>(map)),
-      "r"(ptx::smem_u32(ssrc)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
-      : "memory");
-}
-__device__ __forceinline__ void bulk_commit() {
-  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-__device__ __forceinline__ void bulk_wait_read() {
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-__device__ __forceinline__ void bulk_wait_all() {
-  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-}
-// Stores a shared-memory tile through a tensor map (TMA, asynchronous).
-__device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, const void* ssrc, int c0,
-                                             int c1, int c2, int c3) {
-  asm volatile(
-      "cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
-          reinterpret_cast<uint64_t>(map)),
-      "r"(ptx::smem_u32(ssrc)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
-      : "memory");
-}
-
-
 // One unit of work: the 128 keys [n0, n0+128) of one (batch, key/value head)
 // and the I query tiles (of the group's heads) that see them.
 struct KeyTile {

@@ -1,7 +1,7 @@
-// Thin inline-PTX wrappers for sm_100a: mbarriers (with bounded waits),
-// TMA tensor copies (no multicast), and tcgen05 (TMEM allocation, MMA,
-// commit, TMEM loads/stores, fences), plus the shared-memory matrix and
-// instruction descriptors the MMAs take.
+// Thin inline-PTX wrappers for sm_100a: mbarriers (with bounded waits), TMA
+// tensor copies, stores and reduce-adds (no multicast), and tcgen05 (TMEM
+// allocation, MMA, commit, TMEM loads/stores, fences), plus the shared-memory
+// matrix and instruction descriptors the MMAs take.
 #pragma once
 
 #include <cuda.h>
@@ -102,6 +102,38 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, u
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2),
       "r"(c3)
       : "memory");
+}
+
+// Adds a shared-memory tile into global memory through a tensor map (TMA
+// reduce-add in L2, asynchronous; the tile may be reused after bulk_wait_read).
+__device__ __forceinline__ void tma_reduce_add_4d(const CUtensorMap* map, const void* ssrc, int c0,
+                                                  int c1, int c2, int c3) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.4d.global.shared::cta.add.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(smem_u32(ssrc)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+// Stores a shared-memory tile through a tensor map (TMA, asynchronous; rows
+// outside the tensor are not written).
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, const void* ssrc, int c0,
+                                             int c1, int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(smem_u32(ssrc)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Waits until the committed bulk copies have read their shared-memory sources.
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Waits until the committed bulk copies have completed.
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 // Makes generic-proxy shared-memory writes visible to the async proxy
