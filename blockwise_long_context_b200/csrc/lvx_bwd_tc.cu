@@ -82,8 +82,6 @@ struct BwdLayout {
 struct BwdArgs {
   Problem p;
   float* dq_acc;
-  __nv_bfloat16* dk;
-  __nv_bfloat16* dv;
   unsigned int* err;
   int n_kt;     // key tiles per (batch, kv head)
   int n_qt;     // query tiles per head
@@ -700,8 +698,6 @@ cudaError_t launch(const Problem& p, const void* q, const void* k, const void* v
   BwdArgs a;
   a.p = p;
   a.dq_acc = dq_acc;
-  a.dk = reinterpret_cast<__nv_bfloat16*>(dk);
-  a.dv = reinterpret_cast<__nv_bfloat16*>(dv);
   a.err = device_error_word();
   a.n_kt = (p.S_KV + BKEY - 1) / BKEY;
   a.n_qt = (p.S_Q + BROW - 1) / BROW;
