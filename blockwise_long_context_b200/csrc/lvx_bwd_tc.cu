@@ -275,11 +275,28 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
     } else if (warp == 1) {
       if (lane == 0) {
         // ---------------------------------------------------------------- MMA issuer
-        const uint32_t k_base = ptx::smem_u32(smem + L::OFF_K);
-        const uint32_t v_base = ptx::smem_u32(smem + L::OFF_V);
-        const uint32_t q_base = ptx::smem_u32(smem + L::OFF_Q);
-        const uint32_t do_base = ptx::smem_u32(smem + L::OFF_DO);
-        const uint32_t ds_base = ptx::smem_u32(smem + L::OFF_DS);
+        // Shared-memory descriptors (128-byte swizzle): the high word is the
+        // same for every operand here (sbo 1024, version, swizzle mode), and the
+        // low word is (address >> 4) | (lbo >> 4) << 16.  Only the low words of
+        // the five buffers are kept (K-major form, lbo 16); a stage, K step or
+        // MN-major form (lbo CHUNK) adds a compile-time constant to them.
+        // Shared-memory addresses stay below 2^18, so the 14-bit address field
+        // never carries into lbo.  This keeps the issuing thread, which shares
+        // its sub-partition with three busy warps, at a few instructions per
+        // MMA, within the registers of its warp group.  The empty asm below
+        // marks the five words as changed once per query tile, so that the
+        // compiler derives each descriptor where it is used instead of keeping
+        // every K step's descriptor live across the loop (which spills).
+        uint32_t dK = (ptx::smem_u32(smem + L::OFF_K) >> 4) | (1u << 16);
+        uint32_t dV = (ptx::smem_u32(smem + L::OFF_V) >> 4) | (1u << 16);
+        uint32_t dQ = (ptx::smem_u32(smem + L::OFF_Q) >> 4) | (1u << 16);
+        uint32_t dDO = (ptx::smem_u32(smem + L::OFF_DO) >> 4) | (1u << 16);
+        uint32_t dDS = (ptx::smem_u32(smem + L::OFF_DS) >> 4) | (1u << 16);
+        constexpr uint32_t kMN = ((CHUNK >> 4) - 1u) << 16;   // lbo 16 -> lbo CHUNK
+        auto desc = [](uint32_t lo) {
+          return ((uint64_t)((1024u >> 4) | (1u << 14) | (2u << 29)) << 32) | lo;
+        };
+        constexpr uint32_t kStage16 = L::TILE >> 4;   // one Q / dO stage, in descriptor units
         // Issue order within a key tile: S_0, dP_0, dV_0, then per tile i
         //   S_{i+1}, dK_i, dQ_i, dP_{i+1}, dV_{i+1}.
         // S_{i+1} goes right after dV_i, which reads P_i from the same TMEM
@@ -292,17 +309,16 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
         // for P and dS of its first tile, which the elementwise warps produce
         // only after writing out the previous key tile's dK and dV.
         auto issue_s = [&](int gi) {
-          const uint32_t qs = q_base + (gi & 1) * L::TILE;
+          const uint32_t qs = dQ + (gi & 1) * kStage16;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {   // S^T = K Q^T
-            const uint32_t off = (kk >> 2) * CHUNK + (kk & 3) * 32;
-            ptx::mma_ss(tS, ptx::smem_desc_sw128(k_base + off, 16, 1024),
-                        ptx::smem_desc_sw128(qs + off, 16, 1024), L::IDESC_SS_KK, kk > 0);
+            const uint32_t off = ((kk >> 2) * CHUNK + (kk & 3) * 32) >> 4;
+            ptx::mma_ss(tS, desc(dK + off), desc(qs + off), L::IDESC_SS_KK, kk > 0);
           }
           ptx::mma_commit(s_full);
         };
         auto issue_dp_dv = [&](int gi, bool first_tile) -> bool {
-          const uint32_t dos = do_base + (gi & 1) * L::TILE;
+          const uint32_t dos = dDO + (gi & 1) * kStage16;
           if (!ptx::mbar_wait(&do_full[gi & 1], (gi >> 1) & 1, a.err, kErrTimeoutMma, abort_flag))
             return false;
           ptx::tc_fence_after();
@@ -315,10 +331,9 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
             }
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t off = (kk >> 2) * CHUNK + (kk & 3) * 32;
-              ptx::mma_ss(tdP + 64 * h, ptx::smem_desc_sw128(v_base + off, 16, 1024),
-                          ptx::smem_desc_sw128(dos + off + h * 8192, 16, 1024), L::IDESC_DP_HALF,
-                          kk > 0);
+              const uint32_t off = ((kk >> 2) * CHUNK + (kk & 3) * 32) >> 4;
+              ptx::mma_ss(tdP + 64 * h, desc(dV + off), desc(dos + off + h * (8192 >> 4)),
+                          L::IDESC_DP_HALF, kk > 0);
             }
             ptx::mma_commit(&dp_full[h]);
           }
@@ -327,8 +342,8 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
 #pragma unroll
           for (int kk = 0; kk < BROW / 16; ++kk)   // dV += P^T dO (P^T halves at columns 0 and 64)
             ptx::mma_ts(tdV, tS + (kk >> 2) * 64 + (kk & 3) * 8,
-                        ptx::smem_desc_sw128(dos + kk * 2048, CHUNK, 1024),
-                        L::IDESC_DV, (!first_tile || kk > 0) ? 1u : 0u);
+                        desc(dos + (kMN + kk * (2048 >> 4))), L::IDESC_DV,
+                        (!first_tile || kk > 0) ? 1u : 0u);
           return true;
         };
         int gt = 0, nkv = 0;
@@ -347,6 +362,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
           ok = issue_dp_dv(gt, true);
           for (int i = 0; i < w.I && ok; ++i) {
             const int gi = gt + i;
+            asm volatile("" : "+r"(dK), "+r"(dV), "+r"(dQ), "+r"(dDO), "+r"(dDS));
             if (i + 1 < w.I) {
               ok = ptx::mbar_wait(&q_full[(gi + 1) & 1], ((gi + 1) >> 1) & 1, a.err, kErrTimeoutMma,
                                   abort_flag);
@@ -357,19 +373,18 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
             ok = ptx::mbar_wait(ds_ready, gi & 1, a.err, kErrTimeoutMma, abort_flag);
             if (!ok) break;
             ptx::tc_fence_after();
-            const uint32_t qs = q_base + (gi & 1) * L::TILE;
+            const uint32_t qs = dQ + (gi & 1) * kStage16;
 #pragma unroll
             for (int kk = 0; kk < BROW / 16; ++kk) {   // dK += dS^T Q
-              const uint32_t off = (kk >> 2) * CHUNK + (kk & 3) * 32;
-              ptx::mma_ss(tdK, ptx::smem_desc_sw128(ds_base + off, 16, 1024),
-                          ptx::smem_desc_sw128(qs + kk * 2048, CHUNK, 1024), L::IDESC_DK,
+              const uint32_t off = ((kk >> 2) * CHUNK + (kk & 3) * 32) >> 4;
+              ptx::mma_ss(tdK, desc(dDS + off), desc(qs + (kMN + kk * (2048 >> 4))), L::IDESC_DK,
                           (i > 0 || kk > 0) ? 1u : 0u);
             }
             ptx::mma_commit(&q_empty[gi & 1]);   // Q, LSE, D of this stage are no longer read
 #pragma unroll
             for (int kk = 0; kk < BKEY / 16; ++kk)   // dQ_t = dS K
-              ptx::mma_ss(tdP, ptx::smem_desc_sw128(ds_base + kk * 2048, CHUNK, 1024),
-                          ptx::smem_desc_sw128(k_base + kk * 2048, CHUNK, 1024), L::IDESC_DQ, kk > 0);
+              ptx::mma_ss(tdP, desc(dDS + (kMN + kk * (2048 >> 4))),
+                          desc(dK + (kMN + kk * (2048 >> 4))), L::IDESC_DQ, kk > 0);
             ptx::mma_commit(dq_full);
             if (i + 1 < w.I) ok = issue_dp_dv(gi + 1, false);
             else ptx::mma_commit(kv_free);   // K and V of this key tile are no longer read
