@@ -14,10 +14,12 @@
 //   S^T  = K Q^T        (SS)  -> TMEM [0,128)
 //   dP^T = V dO^T       (SS)  -> TMEM [128,256)
 //   elementwise warps: P^T = exp2(S^T * s*log2e - LSE*log2e) -> bf16 back
-//       into TMEM [0,32) and [64,96); dS^T = P^T o (dP^T - D) -> bf16 into shared memory
+//       into TMEM [0,32) and [64,96); dS^T = P^T o (dP^T - D) -> bf16 into shared
+//       memory, and packed over the dP^T columns already read, TMEM [128,160) and [192,224)
 //   dV  += P^T dO       (TS, A = P^T from TMEM)  -> TMEM [256,256+D)
-//   dK  += dS^T Q       (SS, dS^T read K-major)  -> TMEM [256+D,256+2D)
-//   dQ_t = dS K         (SS, the same dS^T buffer read MN-major) -> TMEM [128,128+D)
+//   dK  += dS^T Q       (TS, A = dS^T from TMEM) -> TMEM [256+D,256+2D)
+//   dQ_t = dS K         (SS, dS^T from shared memory read MN-major) -> TMEM [128,128+D);
+//       issued after dK, so dK has read dS^T before dQ_t overwrites those columns
 //   a drain warpgroup reads dQ_t out of TMEM, releases it, and adds it to the
 //   fp32 dQ accumulator with TMA reduce-add, staged in the tile's dO slot
 //   (idle once dV has run; the next dO load into that slot waits for the
@@ -375,10 +377,9 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
             ptx::tc_fence_after();
             const uint32_t qs = dQ + (gi & 1) * kStage16;
 #pragma unroll
-            for (int kk = 0; kk < BROW / 16; ++kk) {   // dK += dS^T Q
-              const uint32_t off = ((kk >> 2) * CHUNK + (kk & 3) * 32) >> 4;
-              ptx::mma_ss(tdK, desc(dDS + off), desc(qs + (kMN + kk * (2048 >> 4))), L::IDESC_DK,
-                          (i > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < BROW / 16; ++kk) {   // dK += dS^T Q (dS^T halves at columns 0 and 64)
+              ptx::mma_ts(tdK, tdP + (kk >> 2) * 64 + (kk & 3) * 8, desc(qs + (kMN + kk * (2048 >> 4))),
+                          L::IDESC_DK, (i > 0 || kk > 0) ? 1u : 0u);
             }
             ptx::mma_commit(&q_empty[gi & 1]);   // Q, LSE, D of this stage are no longer read
 #pragma unroll
@@ -493,6 +494,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           uint32_t dr[32];
+          uint32_t dsk[16];
           ptx::tmem_ld32(tdP + lane_off + 64 * hf + 32 * half, dr);
           ptx::tmem_wait_ld();
 #pragma unroll
@@ -512,8 +514,13 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
               wd[t] = ptx::pack_bf16x2(e0, e1);
             }
             *reinterpret_cast<uint4*>(ds_smem + ((c8 ^ (j & 7)) << 4)) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+#pragma unroll
+            for (int t = 0; t < 4; ++t) dsk[4 * q8 + t] = wd[t];
           }
+          // dS^T of these 32 rows, packed, over dP^T columns this thread has read
+          ptx::tmem_st16(tdP + lane_off + 64 * hf + 16 * half, dsk);
         }
+        ptx::tmem_wait_st();
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
         ptx::mbar_arrive(ds_ready);
