@@ -44,6 +44,7 @@ static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= 65536 / kThreads * kThr
               "register split exceeds the launch allocation");
 constexpr uint32_t CHUNK = 128 * 128;   // one TMA box: 128 rows x 64 bf16 (128 B), swizzled
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
+constexpr float kRescaleFactor = 256.0f;    // 2^kRescaleThreshold
 constexpr float kLn2 = 0.6931471805599453f;
 
 template <int D>
@@ -197,58 +198,71 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
         // P_t of tile j-1 right after the MMA that reads it; tcgen05.mma ops of
         // one thread execute in issue order, so that read completes first.
         if (T > 0 && ptx::mbar_wait(q_full, 0, a.err, kErrTimeoutMma, abort_flag)) {
-          const uint32_t q_base = ptx::smem_u32(smem + L::OFF_Q);
-          const uint32_t k_base = ptx::smem_u32(smem + L::OFF_K);
-          const uint32_t v_base = ptx::smem_u32(smem + L::OFF_V);
-          auto issue_s = [&](int t, int j) {
-            const int s = j % K_STAGES;
+          // Shared-memory descriptors: only the low words (address >> 4 and lbo)
+          // differ between operands, so the Q, K-stage and V-stage low words are
+          // kept and each K step adds a compile-time offset; the high word
+          // (sbo 1024, version, 128-byte swizzle) is a constant.  The issuing
+          // thread shares its sub-partition with two softmax warps, so every
+          // instruction saved here shortens the PV -> S hand-off on the
+          // critical path.  Addresses stay below 2^18: no carry into lbo.
+          constexpr uint32_t kT16 = L::TILE >> 4;
+          constexpr uint32_t kMN = ((CHUNK >> 4) - 1u) << 16;   // lbo 16 -> lbo CHUNK
+          const uint32_t dQ0 = (ptx::smem_u32(smem + L::OFF_Q) >> 4) | (1u << 16);
+          const uint32_t dK0 = (ptx::smem_u32(smem + L::OFF_K) >> 4) | (1u << 16);
+          const uint32_t dV0 = (ptx::smem_u32(smem + L::OFF_V) >> 4) | (1u << 16);
+          auto desc = [](uint32_t lo) {
+            return ((uint64_t)((1024u >> 4) | (1u << 14) | (2u << 29)) << 32) | lo;
+          };
+          uint32_t dKs = dK0, dVs = dV0;   // this tile's K and V stages
+          auto issue_s = [&](int t) {
+            const uint32_t dq = dQ0 + t * kT16;
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t off = (kk >> 2) * CHUNK + (kk & 3) * 32;
-              const uint64_t da = ptx::smem_desc_sw128(q_base + t * L::TILE + off, 16, 1024);
-              const uint64_t db = ptx::smem_desc_sw128(k_base + s * L::TILE + off, 16, 1024);
-              ptx::mma_ss(tmem + t * 128, da, db, L::IDESC_QK, kk > 0 ? 1u : 0u);
+              const uint32_t off = ((kk >> 2) * CHUNK + (kk & 3) * 32) >> 4;
+              ptx::mma_ss(tmem + t * 128, desc(dq + off), desc(dKs + off), L::IDESC_QK,
+                          kk > 0 ? 1u : 0u);
             }
             ptx::mma_commit(&s_full[t]);
           };
-          auto issue_pv = [&](int t, int j) {
-            const int s = j % V_STAGES;
+          auto issue_pv = [&](int t, uint32_t dv, bool first) {
 #pragma unroll
-            for (int kk = 0; kk < BKV / 16; ++kk) {
-              const uint64_t db =
-                  ptx::smem_desc_sw128(v_base + s * L::TILE + kk * 16 * 128, CHUNK, 1024);
-              ptx::mma_ts(tmem + 256 + t * D, tmem + t * 128 + kk * 8, db, L::IDESC_PV,
-                          (j > 0 || kk > 0) ? 1u : 0u);
-            }
+            for (int kk = 0; kk < BKV / 16; ++kk)
+              ptx::mma_ts(tmem + 256 + t * D, tmem + t * 128 + kk * 8,
+                          desc(dv + (kMN + kk * (2048 >> 4))), L::IDESC_PV,
+                          (!first || kk > 0) ? 1u : 0u);
             ptx::mma_commit(&o_done[t]);
           };
+          uint32_t dVprev = dV0;   // V stage of tile j-1
           bool ok = true;
           for (int j = 0; j < T && ok; ++j) {
             ok = ptx::mbar_wait(&k_full[j % K_STAGES], (j / K_STAGES) & 1, a.err, kErrTimeoutMma,
                                 abort_flag);
             if (!ok) break;
             ptx::tc_fence_after();
-            issue_s(0, j);
+            issue_s(0);
             if (j > 0) {
               // PV1 of the previous tile (its V stage is released afterwards)
               ok = ptx::mbar_wait(&p_full[1], (j - 1) & 1, a.err, kErrTimeoutMma, abort_flag);
               if (!ok) break;
               ptx::tc_fence_after();
-              issue_pv(1, j - 1);
+              issue_pv(1, dVprev, j == 1);
               ptx::mma_commit(&v_empty[(j - 1) % V_STAGES]);
             }
-            issue_s(1, j);
+            issue_s(1);
             ptx::mma_commit(&k_empty[j % K_STAGES]);
             ok = ptx::mbar_wait(&v_full[j % V_STAGES], (j / V_STAGES) & 1, a.err, kErrTimeoutMma,
                                 abort_flag);
             if (ok) ok = ptx::mbar_wait(&p_full[0], j & 1, a.err, kErrTimeoutMma, abort_flag);
             if (!ok) break;
             ptx::tc_fence_after();
-            issue_pv(0, j);
+            issue_pv(0, dVs, j == 0);
+            dVprev = dVs;
+            dKs = (j % K_STAGES == K_STAGES - 1) ? dK0 : dKs + kT16;
+            dVs = (j % V_STAGES == V_STAGES - 1) ? dV0 : dVs + kT16;
           }
           if (ok && ptx::mbar_wait(&p_full[1], (T - 1) & 1, a.err, kErrTimeoutMma, abort_flag)) {
             ptx::tc_fence_after();
-            issue_pv(1, T - 1);
+            issue_pv(1, dVprev, T == 1);
             ptx::mma_commit(&v_empty[(T - 1) % V_STAGES]);
           }
         }
@@ -275,36 +289,49 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
       if (!ok) break;
       ptx::tc_fence_after();
       uint32_t sr[128];
+      // keys 64..127 load while the exponentials of keys 0..63 are computed
       ptx::tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
       ptx::tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      ptx::tmem_wait_ld();
       ptx::tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
       ptx::tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
-      ptx::tmem_wait_ld();
+      // the second wait, after which the compiler must treat keys 64..127 as
+      // written (the load's register outputs are only valid from here on)
+      auto wait_upper = [&]() {
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int i = 64; i < 128; i += 8)
+          asm volatile("" : "+r"(sr[i]), "+r"(sr[i + 1]), "+r"(sr[i + 2]), "+r"(sr[i + 3]),
+                       "+r"(sr[i + 4]), "+r"(sr[i + 5]), "+r"(sr[i + 6]), "+r"(sr[i + 7]));
+      };
       const int key0 = kb0 + BKV * j;
       const bool need_mask = (key0 + BKV > kb1) || (p.causal && key0 + BKV - 1 > row0_tile);
       // Steady state (an unmasked tile once the row has a running maximum): P is
-      // computed with the running maximum straight away, and the tile's maximum
-      // is found in the same pass instead of before it.  Only if it exceeds the
-      // running maximum by more than the threshold (for any row of the warp) is
-      // that P discarded -- nothing has been released yet -- and the tile redone
-      // below with the maximum moved, exactly as a first tile is.
+      // computed with the running maximum straight away, with no pass for the
+      // tile's maximum.  Only if some exponential may exceed 2^threshold (for
+      // any row of the warp) is that P discarded -- nothing has been released
+      // yet -- and the tile redone below with the maximum moved, exactly as a
+      // first tile is.
       bool done = false;
       if (!need_mask && m_ref != -INFINITY) {
         const uint64_t sl2x2 = pk2(sl2, sl2);
         const uint64_t negm2 = pk2(-m_ref, -m_ref);
         uint64_t acc2 = pk2(0.f, 0.f), acc2b = pk2(0.f, 0.f);
-        float mc[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        float xp = -INFINITY;   // largest argument among the FMA-pipe exponentials
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
+          if (c == 2) wait_upper();
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const float s0 = __uint_as_float(sr[32 * c + 2 * i]);
             const float s1 = __uint_as_float(sr[32 * c + 2 * i + 1]);
-            mc[i & 3] = fmax3(mc[i & 3], s0, s1);
             const uint64_t x2 = ffma2(pk2(s0, s1), sl2x2, negm2);
             uint64_t e2;
             if (i % kPolyEvery == kPolyEvery - 1) {
+              float x0, x1;
+              upk2(x2, x0, x1);
+              xp = fmax3(xp, x0, x1);
               e2 = exp2_poly2(x2);
             } else {
               float x0, x1;
@@ -318,13 +345,21 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
           }
           ptx::tmem_st16(tS + 16 * c, pk);
         }
-        const float m_tile = fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3])) * sl2;
-        if (!__any_sync(0xffffffffu, m_tile > m_ref + kRescaleThreshold)) {
-          float a0, a1;
-          upk2(fadd2(acc2, acc2b), a0, a1);
-          l_sum += a0 + a1;
+        // Accepted only if every exponential is at most 2^threshold.  A sum of
+        // positive terms bounds each of them; an SFU exponential of a larger
+        // argument is large or +inf, and a NaN fails the test as well.  The
+        // FMA-pipe exponential is valid only for arguments up to 127, so its
+        // arguments are checked directly.
+        float a0, a1;
+        upk2(fadd2(acc2, acc2b), a0, a1);
+        const float tile_sum = a0 + a1;
+        const bool fits = tile_sum <= kRescaleFactor && xp <= kRescaleThreshold;
+        if (__all_sync(0xffffffffu, fits)) {
+          l_sum += tile_sum;
           done = true;
         }
+      } else {
+        wait_upper();
       }
       if (!done) {
         if (need_mask) {

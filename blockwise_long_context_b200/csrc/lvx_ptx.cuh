@@ -332,12 +332,15 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 // 2^x on the FMA pipe: x = n + f with n = round(x), |f| <= 1/2; 2^f from a
 // cubic fitted by fit_exp2.py (max relative error 7.5e-5, far below the
 // bf16 rounding P receives); n is added to the exponent field.  Adding
-// 1.5 * 2^23 leaves round(x) in the low mantissa bits of t.  x is clamped at
-// -127 so the exponent cannot wrap; callers use it only on unmasked tiles,
-// where the argument is finite.
+// 1.5 * 2^23 leaves round(x) in the low mantissa bits of t.  2^f lies in
+// [2^-1/2, 2^1/2], so its exponent field is 126 or 127: x is clamped at -126,
+// where n + 126 >= 0 and the addition cannot borrow through the sign bit
+// (at -127 it did, giving NaN); below -126 the result is ~2^-126, negligible
+// next to the terms near the row maximum.  Arguments above 127 overflow the
+// exponent field: callers use it where x <= 0, or check x themselves.
 constexpr int kPolyEvery = 4;   // one pair of exponentials in kPolyEvery on the FMA pipe
 __device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -127.f);
+  x = fmaxf(x, -126.f);
   const float t = x + 12582912.f;
   const float f = x - (t - 12582912.f);
   const float p = fmaf(fmaf(fmaf(5.517164990e-02f, f, 2.426111400e-01f), f, 6.932609677e-01f), f,
@@ -349,7 +352,7 @@ __device__ __forceinline__ float exp2_poly(float x) {
 __device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
   float x0, x1;
   upk2(x2, x0, x1);
-  x2 = pk2(fmaxf(x0, -127.f), fmaxf(x1, -127.f));
+  x2 = pk2(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
   const uint64_t magic = pk2(12582912.f, 12582912.f);
   const uint64_t nmagic = pk2(-12582912.f, -12582912.f);
   const uint64_t t = fadd2(x2, magic);

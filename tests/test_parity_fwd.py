@@ -82,6 +82,38 @@ def test_forward_small(case):
         compare(L_g, L_r, w.dtype, f"{name}: L_i", rel_rms=1e-4 if w.dtype == "bf16" else 1e-6)
 
 
+def test_forward_rising_logits_rescale():
+    """Logits that step up from tile to tile inside each key block, so that the
+    running maximum of a row moves after its first tile.  Query head 0 steps by
+    ~12 (log2 units) per 128-key tile: past the rescale threshold of 8, every
+    later tile rescales O.  Head 1 steps by ~6: no exponential exceeds 2^8,
+    but a tile's sum of exponentials does.  Key 262 adds a spike far above the
+    rest (argument > 128 in log2 units for head 0); it sits at a position whose
+    exponential the kernel computes with the FMA-pipe polynomial in the steady
+    state.  All three must match plain attention."""
+    rng = np.random.default_rng(11)
+    B, H, H_kv, d, S_Q, S_KV, n = 1, 2, 1, 128, 130, 1000, 2
+    q = rng.standard_normal((B, S_Q, H, d)) * 0.5
+    k = rng.standard_normal((B, S_KV, H_kv, d)) * 0.5
+    v = rng.standard_normal((B, S_KV, H_kv, d))
+    q[:, :, 0, 0] = 16.0
+    q[:, :, 1, 0] = 8.0
+    block = -(-S_KV // n)
+    k[0, :, 0, 0] = 6.0 * ((np.arange(S_KV) % block) // 128)
+    k[0, 262, 0, 0] = 80.0
+    host = {name: torch.from_numpy(t).to(torch.bfloat16) for name, t in (("q", q), ("k", k), ("v", v))}
+    w = _workload(B, H, H_kv, d, S_Q, S_KV, n, False, "bf16")
+    out, lse, ws = _run(w, host)
+    q, k, v = (host[t].double().numpy() for t in ("q", "k", "v"))
+    o_ref, l_ref = oracle.attention_fwd(q, k, v)
+    compare(out, o_ref, "bf16", "rising logits: O")
+    compare(lse, l_ref, "bf16", "rising logits: LSE", rel_rms=1e-4)
+    O_p, L_p = lvx.fwd_partials_view(ws, n, B, H, S_Q, d)
+    O_r, L_r = oracle.block_partials(q, k, v, n)
+    compare(O_p, np.transpose(O_r, (0, 1, 3, 2, 4)), "bf16", "rising logits: O_i", rel_rms=5e-3)
+    compare(L_p, L_r, "bf16", "rising logits: L_i", rel_rms=1e-4)
+
+
 def test_merge_entry_point_matches_oracle():
     rng = np.random.default_rng(3)
     n, B, H, S_Q, d = 5, 2, 3, 77, 128
