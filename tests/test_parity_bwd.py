@@ -77,6 +77,38 @@ def test_backward_small(case):
     _invariants(w, host, dk, dv, tol=1e-2 if w.dtype == "bf16" else 1e-5)
 
 
+def test_backward_far_below_the_maximum():
+    """Keys whose logits lie far below the row's log-sum-exp: P = exp2(x) with
+    x < -126 (log2 units), where the kernel's FMA-pipe exponential is at its
+    clamp.  Query head 0 sees a spike at key 262 ~88 natural-log units above
+    every other key, so most of its arguments are there; head 1 sees the
+    same keys through a logit ramp of ~2 per 128-key tile, which gives the
+    compared tensors gradients of ordinary size."""
+    rng = np.random.default_rng(12)
+    B, H, H_kv, d, S_Q, S_KV = 1, 2, 1, 128, 130, 1000
+    q = rng.standard_normal((B, S_Q, H, d)) * 0.5
+    k = rng.standard_normal((B, S_KV, H_kv, d)) * 0.5
+    v = rng.standard_normal((B, S_KV, H_kv, d))
+    do = rng.standard_normal((B, S_Q, H, d)) * 0.05   # dV of the spike key stays ~1
+    q[:, :, 0, 0], q[:, :, 1, 0] = 16.0, 4.0
+    q[:, :, 0, 1], q[:, :, 1, 1] = 16.0, 0.0
+    k[0, :, 0, 0] = 6.0 * ((np.arange(S_KV) % 500) // 128)
+    k[0, :, 0, 1] = 0.0
+    k[0, 262, 0, 1] = 80.0
+    host = {name: torch.from_numpy(t).to(torch.bfloat16)
+            for name, t in (("q", q), ("k", k), ("v", v), ("do", do))}
+    w = _workload(B, H, H_kv, d, S_Q, S_KV, False, "bf16")
+    out, lse, dq, dk, dv = _run(w, host)
+    for name, t in (("dQ", dq), ("dK", dk), ("dV", dv)):
+        assert torch.isfinite(t.float()).all(), f"{name} not finite"
+    q, k, v, do = (host[t].double().numpy() for t in ("q", "k", "v", "do"))
+    dq_r, dk_r, dv_r = oracle.attention_bwd(q, k, v, do)
+    compare(dq, dq_r, "bf16", "far below: dQ")
+    compare(dk, dk_r, "bf16", "far below: dK")
+    compare(dv, dv_r, "bf16", "far below: dV")
+    _invariants(w, host, dk, dv)
+
+
 @pytest.mark.parametrize("cfg", ["C2", "C4", "C3"])
 def test_backward_full_size_sampled(cfg):
     w = inputs.WORKLOADS[cfg]
