@@ -39,7 +39,7 @@ _SIGS = {
     "lvx_attn_fwd_workspace": ([_c_int] * 8 + [_c_int], _c_size),
     "lvx_attn_fwd": ([_vp] * 5 + [_c_int] * 8 + [_c_int, _c_float, _vp, _c_size, _vp], _c_int),
     "lvx_merge_partials": ([_vp] * 4 + [_c_int] * 5 + [_c_int, _vp], _c_int),
-    "lvx_attn_fwd_partials": ([_vp] * 5 + [_c_int] * 7 + [_c_int, _c_float, _vp], _c_int),
+    "lvx_attn_fwd_partials": ([_vp] * 5 + [_c_int] * 8 + [_c_int, _c_float, _vp], _c_int),
     "lvx_attn_fwd_noalloc": ([_vp] * 5 + [_c_int] * 8 + [_c_int, _c_float, _vp], _c_int),
     "lvx_attn_bwd_workspace": ([_c_int] * 7 + [_c_int], _c_size),
     "lvx_attn_bwd": ([_vp] * 9 + [_c_int] * 7 + [_c_int, _c_float, _vp, _c_size, _vp], _c_int),
@@ -127,14 +127,16 @@ def lvx_attn_fwd_noalloc(q, k, v, out, lse, n_blocks: int, causal: bool = False,
                                       _stream(stream)), "lvx_attn_fwd_noalloc")
 
 
-def lvx_attn_fwd_partials(q, k, v, o_parts, l_parts, scale: float = 0.0, stream=None) -> None:
+def lvx_attn_fwd_partials(q, k, v, o_parts, l_parts, scale: float = 0.0, stream=None,
+                          causal: bool = False) -> None:
     """q [B,S_Q,H,d], k/v [B,S_KV,H_kv,d] (a shard of the keys/values) ->
-    o_parts [n,B,H,S_Q,d] fp32, l_parts [n,B,H,S_Q] fp32; n is o_parts.shape[0]."""
+    o_parts [n,B,H,S_Q,d] fp32, l_parts [n,B,H,S_Q] fp32; n is o_parts.shape[0].
+    causal: key j visible to row r iff j <= r (S_Q == S_KV)."""
     B, S_Q, H, d = q.shape
     S_KV, H_kv = k.shape[1], k.shape[2]
     n = o_parts.shape[0]
     _check(lib().lvx_attn_fwd_partials(_ptr(q), _ptr(k), _ptr(v), _ptr(o_parts), _ptr(l_parts), B, H,
-                                       H_kv, S_Q, S_KV, d, n, _dt(q), float(scale),
+                                       H_kv, S_Q, S_KV, d, n, int(bool(causal)), _dt(q), float(scale),
                                        _stream(stream)), "lvx_attn_fwd_partials")
 
 

@@ -120,17 +120,18 @@ lvx_status lvx_attn_fwd(const void* q, const void* k, const void* v, void* out, 
 
 lvx_status lvx_attn_fwd_partials(const void* q, const void* k, const void* v, float* O_parts,
                                  float* L_parts, int B, int H, int H_kv, int S_Q, int S_KV, int d,
-                                 int n_blocks, lvx_dtype dt, float scale, lvx_stream stream) {
-  lvx_status st = check_shapes(B, H, H_kv, S_Q, S_KV, d, n_blocks, 0, dt);
+                                 int n_blocks, int causal, lvx_dtype dt, float scale,
+                                 lvx_stream stream) {
+  lvx_status st = check_shapes(B, H, H_kv, S_Q, S_KV, d, n_blocks, causal, dt);
   if (st != LVX_OK) return st;
   if (!q || !k || !v || !O_parts || !L_parts) return LVX_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(O_parts) || !aligned16(L_parts))
     return LVX_ERR_INVALID_ARG;
   if (!(scale == scale)) return LVX_ERR_INVALID_ARG;   // NaN scale
-  const Problem p = make_problem(B, H, H_kv, S_Q, S_KV, d, n_blocks, 0, scale);
+  const Problem p = make_problem(B, H, H_kv, S_Q, S_KV, d, n_blocks, causal ? 1 : 0, scale);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  // with a partials buffer the kernels write (O_i, L_i) of every block and
-  // never touch the final-output pointers
+  // with a partials buffer the kernels write (O_i, L_i) of every block (with a
+  // mask: of every block a row sees) and never touch the final-output pointers
   cudaError_t e;
   if (dt == LVX_BF16 && tc_fwd_supported(p))
     e = launch_fwd_tc(p, q, k, v, nullptr, nullptr, O_parts, L_parts, s);

@@ -136,18 +136,25 @@ lvx_status lvx_attn_fwd_noalloc(const void* q, const void* k, const void* v, voi
  * own, for callers that merge elsewhere -- in LV-XAttn each worker keeps one
  * stationary shard of the keys and values and its partials are combined with
  * the other workers' (LV-XAttn review page, "The reading" and Figure 3 /
- * Algorithm 1; the rescaling is lvx_merge_partials).
+ * Algorithm 1; the rescaling is lvx_merge_partials); in Ring Attention each
+ * worker computes the partial of its query block against the key/value block
+ * it holds at each ring step (Ring Attention with Blockwise Transformers
+ * page, abstract; LV-XAttn review page, "Core claim").
  *   q [B,S_Q,H,d], k, v [B,S_KV,H_kv,d] (device, dtype dt): the caller's shard
  *   of the keys and values, cut into n_blocks blocks as lvx_attn_fwd cuts them.
  *   O_parts [n_blocks, B, H, S_Q, d] float32 and L_parts [n_blocks, B, H, S_Q]
  *   float32 (device, caller-owned, 16-byte aligned): the normalised partial
  *   outputs and their natural-log log-sum-exp; an empty block writes (0, -inf).
- * Non-causal only (a shard of a cross-attention key sequence): the same
- * constraints and errors as lvx_attn_fwd with causal = 0 and no workspace.
+ * causal = 1 (S_Q == S_KV, the diagonal block of a self-attention): key j is
+ * visible to query row r iff j <= r.  With n_blocks > 1, the partial of block
+ * i is written only for the rows that see some key of it (r >= i * block
+ * length); the other rows of O_parts / L_parts are left as they were.
+ * The same constraints and errors as lvx_attn_fwd without a workspace.
  */
 lvx_status lvx_attn_fwd_partials(const void* q, const void* k, const void* v, float* O_parts,
                                  float* L_parts, int B, int H, int H_kv, int S_Q, int S_KV, int d,
-                                 int n_blocks, lvx_dtype dt, float scale, lvx_stream stream);
+                                 int n_blocks, int causal, lvx_dtype dt, float scale,
+                                 lvx_stream stream);
 
 /*
  * Merge of block partials on its own (the rescaling step of lvx_attn_fwd),

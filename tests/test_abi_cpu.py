@@ -107,18 +107,18 @@ def test_bwd_and_kv_reject_invalid_arguments():
 
 def _parts(**kw):
     a = dict(q=P16, k=P16, v=P16, O=P16, L=P16, B=1, H=2, H_kv=1, S_Q=4, S_KV=4, d=64, n=1,
-             dt=lvx.LVX_BF16, scale=0.0)
+             causal=0, dt=lvx.LVX_BF16, scale=0.0)
     a.update(kw)
     return lvx.lib().lvx_attn_fwd_partials(a["q"], a["k"], a["v"], a["O"], a["L"], a["B"], a["H"],
-                                           a["H_kv"], a["S_Q"], a["S_KV"], a["d"], a["n"], a["dt"],
-                                           a["scale"], None)
+                                           a["H_kv"], a["S_Q"], a["S_KV"], a["d"], a["n"],
+                                           a["causal"], a["dt"], a["scale"], None)
 
 
 @pytest.mark.parametrize("kw,code", [
     (dict(O=None), INVALID), (dict(L=None), INVALID), (dict(v=None), INVALID),
     (dict(O=24), INVALID), (dict(n=0), INVALID), (dict(n=5), INVALID),
     (dict(H=3, H_kv=2), INVALID), (dict(d=136), UNSUPPORTED), (dict(dt=7), UNSUPPORTED),
-    (dict(scale=float("nan")), INVALID),
+    (dict(scale=float("nan")), INVALID), (dict(causal=1, S_KV=8), UNSUPPORTED),
 ])
 def test_fwd_partials_rejects_invalid_arguments(kw, code):
     assert _parts(**kw) == code
