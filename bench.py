@@ -489,6 +489,100 @@ def run_gpu(a):
         dist.destroy_process_group()
 
 
+def run_ring(a):
+    """Ring Attention (pass-KV), the busiest rank of a ``--ring W`` ring on one GPU.
+
+    Rank W-1 under the causal mask (it computes W-1 full blocks and the diagonal;
+    any rank without the mask): its block partials, their merge and its block
+    gradients, with the library's kernels, timed with CUDA events.  ``value`` is
+    that rank's measured TFLOP/s.  ``projection`` divides the whole problem's
+    FLOPs by the busiest rank's time: what W GPUs would reach if the key/value
+    transfers are hidden, which ``comm`` checks against the measured 770 GB/s
+    NVLink peer-copy bandwidth.  Nothing crosses a GPU boundary in this run."""
+    import torch
+    from blockwise_long_context_b200 import inputs
+    from blockwise_long_context_b200 import binding as lvx
+    from blockwise_long_context_b200.ring import (DIAG, SKIP, kernel_block_grad, kernel_merge,
+                                                  kernel_partial, ring_schedule, shard_bounds)
+    W = a.ring
+    w = inputs.WORKLOADS[a.workload].scaled(backward=True, d_embed=0)
+    if a.s_kv:
+        w = w.scaled(S_KV=a.s_kv, S_Q=a.s_kv if w.causal else w.S_Q)
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    d = inputs.make_device(w, tensors=("q", "k", "v", "do"), device=dev)
+    r = W - 1 if w.causal else 0
+    qlo, qhi = shard_bounds(w.S_Q, W, r)
+    q_r, do_r = d["q"][:, qlo:qhi].contiguous(), d["do"][:, qlo:qhi].contiguous()
+    sched = [ring_schedule(r, W, s_, w.causal) for s_ in range(W)]
+    blocks = {}
+    for src, mode in sched:
+        if mode != SKIP:
+            lo, hi = shard_bounds(w.S_KV, W, src)
+            blocks[src] = (d["k"][:, lo:hi].contiguous(), d["v"][:, lo:hi].contiguous())
+    del d
+    partial, grad, merge = kernel_partial(), kernel_block_grad(), kernel_merge(q_r)
+    B, S_r, H, hd = q_r.shape
+    o_parts = torch.zeros((W, B, H, S_r, hd), dtype=torch.float32, device=dev)
+    l_parts = torch.full((W, B, H, S_r), float("-inf"), dtype=torch.float32, device=dev)
+    dq = torch.zeros(q_r.shape, dtype=torch.float32, device=dev)
+    acc = {src: (torch.zeros(kv[0].shape, dtype=torch.float32, device=dev),
+                 torch.zeros(kv[1].shape, dtype=torch.float32, device=dev)) for src, kv in blocks.items()}
+
+    def rank_step():
+        for s_, (src, mode) in enumerate(sched):
+            if mode != SKIP:
+                partial(q_r, *blocks[src], o_parts[s_:s_ + 1], l_parts[s_:s_ + 1], mode == DIAG)
+        out, lse = merge(o_parts, l_parts)
+        for src, mode in sched:
+            if mode != SKIP:
+                gq, gk, gv = grad(q_r, *blocks[src], out, lse, do_r, mode == DIAG)
+                dq.add_(gq); acc[src][0].add_(gk); acc[src][1].add_(gv)
+
+    rank_flops = 0.0
+    for src, mode in sched:
+        if mode == SKIP:
+            continue
+        S_k = blocks[src][0].shape[1]
+        pairs = S_r * (S_r + 1) / 2 if mode == DIAG else S_r * S_k
+        rank_flops += 3.5 * 4.0 * B * H * pairs * hd
+    for _ in range(max(a.warmup, 3)):
+        rank_step()
+    torch.cuda.synchronize()
+    lvx.lvx_last_device_error()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(0)
+    clocks.start()
+    time.sleep(0.3)
+    e0.record()
+    for _ in range(a.steps):
+        rank_step()
+    e1.record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    lvx.lvx_last_device_error()
+    ms = e0.elapsed_time(e1) / a.steps
+    total = w.fwd_flops() + w.bwd_flops()
+    kv_step_bytes = 2 * B * (w.S_KV // W) * w.H_kv * w.d * 2
+    line = {
+        "metric": f"Ring Attention fwd+bwd, busiest rank of a {W}-rank ring, on one GPU",
+        "value": rank_flops / ms / 1e9, "unit": "TFLOP/s", "n_gpus": 1, "steps": a.steps,
+        "warmup": max(a.warmup, 3), "ms_per_rank_step": ms, "higher_is_better": True,
+        "dtype": "bf16", "data": "synthetic (seeded Gaussian)",
+        "config": {"workload": f"{w.name}: ring of {W} ranks, rank {r} (the busiest)", "B": w.B,
+                   "H": w.H, "H_kv": w.H_kv, "d": w.d, "S_Q": w.S_Q, "S_KV": w.S_KV,
+                   "causal": w.causal, "blocks_computed": sum(m != SKIP for _, m in sched)},
+        "rank_flops": rank_flops,
+        "projection": {"ring_tflops": total / ms / 1e9, "per_gpu_tflops": total / ms / 1e9 / W,
+                       "assumes": f"{W} GPUs, key/value transfers hidden behind the compute"},
+        "comm": {"kv_bytes_per_step": kv_step_bytes,
+                 "ms_per_step_at_770_GBps": kv_step_bytes / 770e9 * 1e3,
+                 "compute_ms_per_step": ms / sum(m != SKIP for _, m in sched)},
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -501,9 +595,13 @@ def main():
                     help="also run the gradients of the K/V recomputation (dW_k, dW_v, dy) each step")
     ap.add_argument("--s-kv", type=int, default=0,
                     help="override S_KV (smaller case of the same workload, for profiler captures)")
+    ap.add_argument("--ring", type=int, default=0,
+                    help="time the busiest rank of a Ring Attention ring of this many ranks (one GPU)")
     a = ap.parse_args()
     if a.impl == "reference":
         run_reference(a)
+    elif a.ring:
+        run_ring(a)
     else:
         run_gpu(a)
 
