@@ -17,7 +17,8 @@ INVALID, UNSUPPORTED, WORKSPACE = 1, 2, 3
 
 
 def _declared():
-    src = open(HEADER).read()
+    with open(HEADER) as f:
+        src = f.read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     return sorted(set(re.findall(r"\b(lvx_[a-z_0-9]+)\s*\(", src)))
 

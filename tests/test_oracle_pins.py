@@ -35,7 +35,8 @@ def _qkv(B=2, S_Q=5, S_KV=13, H=4, H_kv=2, d=8, seed=0, std=1.0):
 # ---------------------------------------------------------------- closed forms
 
 def test_golden_two_keys():
-    g = json.load(open(os.path.join(GOLDEN, "two_key_closed_form.json")))
+    with open(os.path.join(GOLDEN, "two_key_closed_form.json")) as f:
+        g = json.load(f)
     q = np.array(g["q"])[None, :, None, :]
     k = np.array(g["k"])[None, :, None, :]
     v = np.array(g["v"])[None, :, None, :]
@@ -50,7 +51,8 @@ def test_golden_two_keys():
 
 
 def test_golden_causal_uniform():
-    g = json.load(open(os.path.join(GOLDEN, "causal_uniform_closed_form.json")))
+    with open(os.path.join(GOLDEN, "causal_uniform_closed_form.json")) as f:
+        g = json.load(f)
     v = np.array(g["v"])[None, :, None, :]
     S, d = v.shape[1], v.shape[3]
     q = np.zeros((1, S, 1, d))
