@@ -9,10 +9,19 @@ Here every rank computes its shard's block partials for all query rows with
 ``lvx_attn_fwd_partials`` (the library's kernels), the ranks exchange them in
 one all-gather over ``torch.distributed`` (NCCL over NVLink between GPUs), and
 every rank merges all partials with ``lvx_merge_partials``.  This is the
-all-gather form of the exchange; the pages' ring of (Q, O, L) moves the same
-(d + 1) * 4 bytes per (head, query row) per rank, in n rounds.  The result is
-replicated on every rank.  Only the gather is communication; both compute
-steps run in the library's CUDA kernels, and there is no CPU path.
+all-gather form of the exchange, and its result is replicated on every rank.
+
+``xattn_forward_ring`` is the ring form: the query rows are sharded too, each
+rank's query block travels around the ring (its transfer overlapping the
+partial computed on the block held), and each partial goes straight back to
+the query block's owner, which merges the W partials of its rows once.  The
+pages rescale the travelling (O, L) at every hop; merging all partials at the
+owner moves the same bytes (one partial per round per rank) and gives the
+same result up to the order of the rescaling.  Each rank ends with the output
+of its own query rows.
+
+Only the transfers are communication; every compute step runs in the
+library's CUDA kernels, and there is no CPU path.
 """
 
 from __future__ import annotations
@@ -82,3 +91,51 @@ def xattn_forward_sharded(q: torch.Tensor, k_shard: torch.Tensor, v_shard: torch
     lse = torch.empty(B, H, S_Q, dtype=torch.float32, device=q.device)
     lvx.lvx_merge_partials(o_all, l_all, out, lse, stream)
     return out, lse
+
+
+def run_xattn_ring(q, k, v, partial_fn, merge_fn, exchange):
+    """LV-XAttn's rotation of the query blocks (LV-XAttn review page, "What
+    carries the argument"; Figure 3 / Algorithm 1).  This rank keeps k, v
+    [B, S_kv_r, H_kv, d]; q [B, S_r, H, d] is its query block.  In round s it
+    holds the query block of rank (r - s) mod W, starts passing it on, computes
+    that block's partial against k, v with ``partial_fn`` (signature as in
+    ``ring.run_ring_forward``) and sends the partial to the block's owner,
+    receiving its own block's partial from rank (r + s) mod W.  ``merge_fn``
+    merges the W partials of this rank's rows."""
+    world, rank = exchange.world, exchange.rank
+    B, S_r, H, d = q.shape
+    q_len = exchange.lengths(S_r, q.device)
+    o_parts = torch.zeros((world, B, H, S_r, d), dtype=torch.float32, device=q.device)
+    l_parts = torch.full((world, B, H, S_r), float("-inf"), dtype=torch.float32, device=q.device)
+    q_cur, in_flight = q, []
+    for s in range(world):
+        owner = (rank - s) % world
+        handle = None
+        if s + 1 < world:
+            handle = exchange.start([q_cur], q_len[(rank - s - 1) % world])
+        if s == 0:
+            partial_fn(q_cur, k, v, o_parts[0:1], l_parts[0:1], False)
+        else:
+            S_o = q_cur.shape[1]
+            o_p = torch.zeros((1, B, H, S_o, d), dtype=torch.float32, device=q.device)
+            l_p = torch.full((1, B, H, S_o), float("-inf"), dtype=torch.float32, device=q.device)
+            partial_fn(q_cur, k, v, o_p, l_p, False)
+            in_flight.append(exchange.exchange([o_p, l_p], owner, [o_parts[s], l_parts[s]],
+                                               (rank + s) % world))
+        if handle is not None:
+            q_cur = exchange.finish(handle)[0]
+    for h in in_flight:
+        exchange.finish(h)
+    return merge_fn(o_parts, l_parts)
+
+
+def xattn_forward_ring(q, k_shard, v_shard, group=None, scale: float = 0.0, stream=None):
+    """Cross-attention with the query rows and the key/value sequence both
+    sharded across the ranks of ``group`` (rank r holds rows
+    ``shard_bounds(S, W, r)`` of each) -> out [B, S_r, H, d], lse [B, H, S_r]
+    float32 for this rank's query rows.  Non-causal."""
+    if not q.is_cuda:
+        raise RuntimeError("xattn_forward_ring runs in the CUDA library; q must be on a GPU")
+    from .ring import RingExchange, kernel_merge, kernel_partial
+    return run_xattn_ring(q, k_shard, v_shard, kernel_partial(scale, stream),
+                          kernel_merge(q, stream), RingExchange(group))

@@ -80,28 +80,38 @@ class RingExchange:
         dist.all_gather(all_n, mine, group=self.group)
         return [int(t.item()) for t in all_n]
 
+    def exchange(self, sends: Sequence[torch.Tensor], dst: int,
+                 recvs: Sequence[torch.Tensor], src: int):
+        """Starts sending ``sends`` to rank ``dst`` and receiving into ``recvs``
+        (contiguous, preallocated) from rank ``src``, as one batch; returns a
+        handle for ``finish``.  Every rank must post its matching half."""
+        # empty tensors are not sent: both sides know every shard's length, so
+        # they leave out the same transfers
+        sends = [t.contiguous() for t in sends if t.numel() > 0]
+        ops = [dist.P2POp(dist.isend, t, self._global(dst), self.group) for t in sends]
+        ops += [dist.P2POp(dist.irecv, r, self._global(src), self.group) for r in recvs
+                if r.numel() > 0]
+        works = dist.batch_isend_irecv(ops) if ops else []
+        return list(recvs), works, sends   # the send buffers stay referenced until finish
+
     def start(self, tensors: Sequence[torch.Tensor], seq_len: Optional[int] = None):
-        """Sends ``tensors`` on; the ones received have the same shapes except
-        dimension 1, which is ``seq_len`` (the length of the incoming block)."""
+        """Sends ``tensors`` to the next rank; the ones received from the previous
+        rank have the same shapes except dimension 1, which is ``seq_len`` (the
+        length of the incoming block)."""
         if self.world == 1:
             return list(tensors), []
-        nxt = self._global((self.rank + 1) % self.world)
-        prv = self._global((self.rank - 1) % self.world)
         recv = []
         for t in tensors:
             shape = list(t.shape)
             if seq_len is not None:
                 shape[1] = seq_len
             recv.append(torch.empty(shape, dtype=t.dtype, device=t.device))
-        ops = []
-        for t, r in zip(tensors, recv):
-            ops.append(dist.P2POp(dist.isend, t.contiguous(), nxt, self.group))
-            ops.append(dist.P2POp(dist.irecv, r, prv, self.group))
-        return recv, dist.batch_isend_irecv(ops)
+        return self.exchange(tensors, (self.rank + 1) % self.world, recv,
+                             (self.rank - 1) % self.world)
 
     @staticmethod
     def finish(handle) -> List[torch.Tensor]:
-        recv, works = handle
+        recv, works = handle[0], handle[1]
         for w in works:
             w.wait()
         return recv

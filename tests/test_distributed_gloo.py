@@ -4,7 +4,10 @@ The distributed forward keeps one key/value shard per rank, gathers every
 rank's block partials (O_i, L_i) and merges them.  These tests check the host
 side of that on CPU: the shard partition, and that the partials of each
 rank's shard, gathered over two and three gloo ranks by ``gather_partials``
-(the function the GPU path uses), merge to exact attention on every rank.
+(the function the GPU path uses), merge to exact attention on every rank;
+and that in the ring form (``run_xattn_ring``: query rows sharded too, query
+blocks travelling, partials returned to their owner) every rank ends with
+exact attention for its own rows, over two to four ranks.
 The partials and the merge here come from the fp64 oracle -- the library's
 kernels need a GPU; ``tests/test_parity_distributed.py`` runs those.
 """
@@ -89,3 +92,59 @@ def test_gathered_shard_partials_merge_to_attention(world, n_local):
     # every rank gathered the same tensors
     sums = {r: v[2] for r, v in res.items()}
     assert len(set(sums.values())) == 1
+
+
+def _ring_worker(rank, world, port, results):
+    """LV-XAttn's ring form: query rows and keys both sharded, query blocks
+    travelling, partials sent back to their owner and merged there."""
+    import datetime
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    import oracle
+    from blockwise_long_context_b200.distributed import run_xattn_ring, shard_bounds
+    from blockwise_long_context_b200.ring import RingExchange
+    rng = np.random.default_rng(9)
+    B, S_Q, H, H_kv, d, S_KV = 2, 11, 4, 2, 8, 31      # uneven shards for 2 and 3 ranks
+    if world == 4:
+        S_Q = 9                                        # query shards 3, 3, 3, 0
+    q = rng.standard_normal((B, S_Q, H, d))
+    k = rng.standard_normal((B, S_KV, H_kv, d))
+    v = rng.standard_normal((B, S_KV, H_kv, d))
+    qlo, qhi = shard_bounds(S_Q, world, rank)
+    klo, khi = shard_bounds(S_KV, world, rank)
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).float()
+
+    def partial(qq, kk, vv, o, l, diagonal):
+        if qq.shape[1] == 0 or kk.shape[1] == 0:
+            return
+        O, L = oracle.block_partials(qq.double().numpy(), kk.double().numpy(), vv.double().numpy(), 1)
+        o.copy_(torch.from_numpy(np.transpose(O, (0, 1, 3, 2, 4))))
+        l.copy_(torch.from_numpy(L))
+
+    def merge(o, l):
+        out, lse = oracle.merge_partials(np.transpose(o.double().numpy(), (0, 1, 3, 2, 4)),
+                                         l.double().numpy())
+        return torch.from_numpy(out), torch.from_numpy(lse)
+
+    out, lse = run_xattn_ring(t(q[:, qlo:qhi]), t(k[:, klo:khi]), t(v[:, klo:khi]), partial, merge,
+                              RingExchange())
+    o_ref, l_ref = oracle.attention_fwd(*(t(a).double().numpy() for a in (q, k, v)))
+    err = lambda a, b: float(np.abs(a - b).max()) if b.size else 0.0   # empty shard: nothing
+    results[rank] = (err(out.numpy(), o_ref[:, qlo:qhi]), err(lse.numpy(), l_ref[:, :, qlo:qhi]))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3, 4])
+def test_ring_form_query_blocks_travel_and_partials_merge_at_their_owner(world):
+    port = _free_port()
+    with mp.Manager() as m:
+        results = m.dict()
+        mp.spawn(_ring_worker, args=(world, port, results), nprocs=world, join=True)
+        res = dict(results)
+    assert sorted(res) == list(range(world))
+    for rank, (eo, el) in res.items():
+        assert eo < 1e-5 and el < 1e-5, (rank, eo, el)

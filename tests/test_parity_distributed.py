@@ -110,3 +110,56 @@ def test_sharded_forward_through_torch_distributed():
     o_ref, l_ref = _oracle(host)
     compare(out, o_ref, "bf16", "torch.distributed: O")
     compare(lse, l_ref, "bf16", "torch.distributed: LSE", rel_rms=1e-4)
+
+
+@pytest.mark.parametrize("world,S_Q,S_KV", [(2, 300, 1024), (3, 300, 1000), (4, 9, 999)])
+def test_ring_form_emulated_ranks(world, S_Q, S_KV):
+    """LV-XAttn's ring form with the query rows sharded too: in round s rank r
+    computes the partial of rank (r - s)'s query block against its own shard,
+    with the same step functions the distributed driver uses; each owner merges
+    its W partials.  (4, 9, ...) leaves one rank without query rows."""
+    from blockwise_long_context_b200.ring import kernel_merge, kernel_partial
+    w, host = _problem(1, 8, 2, 128, S_Q, S_KV)
+    dev = {t: x.cuda() for t, x in host.items()}
+    qb = [shard_bounds(S_Q, world, r) for r in range(world)]
+    kb = [shard_bounds(S_KV, world, r) for r in range(world)]
+    q = [dev["q"][:, lo:hi].contiguous() for lo, hi in qb]
+    k = [dev["k"][:, lo:hi].contiguous() for lo, hi in kb]
+    v = [dev["v"][:, lo:hi].contiguous() for lo, hi in kb]
+    partial = kernel_partial()
+    parts = []
+    for o in range(world):
+        S_o = q[o].shape[1]
+        parts.append((torch.zeros(world, w.B, w.H, S_o, w.d, dtype=torch.float32, device="cuda"),
+                      torch.full((world, w.B, w.H, S_o), float("-inf"), device="cuda")))
+    for r in range(world):
+        for s in range(world):
+            o = (r - s) % world
+            partial(q[o], k[r], v[r], parts[o][0][s:s + 1], parts[o][1][s:s + 1], False)
+    outs, lses = zip(*(kernel_merge(q[o])(*parts[o]) for o in range(world)))
+    lvx.lvx_last_device_error()
+    torch.cuda.synchronize()
+    o_ref, l_ref = _oracle(host)
+    compare(torch.cat(outs, 1), o_ref, "bf16", f"ring form x{world}: O")
+    compare(torch.cat(lses, 2), l_ref, "bf16", f"ring form x{world}: LSE", rel_rms=1e-4)
+
+
+def test_ring_form_through_torch_distributed():
+    """xattn_forward_ring through a one-rank NCCL group."""
+    import torch.distributed as dist
+    from blockwise_long_context_b200.distributed import xattn_forward_ring
+    w, host = _problem(2, 4, 2, 128, 256, 1500)
+    dev = {t: x.cuda() for t, x in host.items()}
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    os.environ["MASTER_PORT"] = str(_free_port())
+    dist.init_process_group("nccl", rank=0, world_size=1, timeout=datetime.timedelta(seconds=60),
+                            device_id=torch.device("cuda", 0))
+    try:
+        out, lse = xattn_forward_ring(dev["q"], dev["k"], dev["v"])
+        lvx.lvx_last_device_error()
+        torch.cuda.synchronize()
+    finally:
+        dist.destroy_process_group()
+    o_ref, l_ref = _oracle(host)
+    compare(out, o_ref, "bf16", "ring form, torch.distributed: O")
+    compare(lse, l_ref, "bf16", "ring form, torch.distributed: LSE", rel_rms=1e-4)

@@ -2,7 +2,7 @@
 
 ``run_ring_forward`` / ``run_ring_backward`` (the drivers the GPU path uses)
 move each key/value block, and in the backward its dK/dV accumulators, around
-two and three gloo ranks.  The per-block steps here are CPU stand-ins: the
+two to four gloo ranks (with four, one rank's shard is empty).  The per-block steps here are CPU stand-ins: the
 forward partial is the oracle's block partial, and the block gradient is the
 textbook blockwise gradient with the global log-sum-exp (written out below).
 The assembled outputs and gradients must equal the oracle's full attention
@@ -83,6 +83,8 @@ def _worker(rank, world, port, causal, results):
     rng = np.random.default_rng(21)                  # the same full problem on every rank
     B, H, H_kv, d = 2, 4, 2, 8
     S_Q, S_KV = (23, 23) if causal else (13, 29)
+    if world == 4:                                   # a trailing shard is empty: 3, 3, 3, 0
+        S_Q, S_KV = (9, 9) if causal else (9, 29)
     q = rng.standard_normal((B, S_Q, H, d))
     k = rng.standard_normal((B, S_KV, H_kv, d))
     v = rng.standard_normal((B, S_KV, H_kv, d))
@@ -94,6 +96,8 @@ def _worker(rank, world, port, causal, results):
     q_r, k_r, v_r, do_r = t(q[:, qlo:qhi]), t(k[:, klo:khi]), t(v[:, klo:khi]), t(do[:, qlo:qhi])
 
     def partial(qq, kk, vv, o, l, diagonal):
+        if qq.shape[1] == 0 or kk.shape[1] == 0:
+            return
         O, L = oracle.block_partials(qq.double().numpy(), kk.double().numpy(), vv.double().numpy(),
                                      1, causal=diagonal)
         o.copy_(torch.from_numpy(np.transpose(O, (0, 1, 3, 2, 4))))
@@ -117,7 +121,8 @@ def _worker(rank, world, port, causal, results):
     qf, kf, vf, dof = (t(a).double().numpy() for a in (q, k, v, do))   # the float32 inputs
     o_ref, l_ref = oracle.attention_fwd(qf, kf, vf, causal=causal)
     dq_ref, dk_ref, dv_ref = oracle.attention_bwd(qf, kf, vf, dof, causal=causal)
-    rel = lambda a, b: float(np.abs(a - b).max() / max(np.abs(b).max(), 1e-30))
+    rel = lambda a, b: (float(np.abs(a - b).max() / max(np.abs(b).max(), 1e-30)) if b.size
+                        else 0.0)   # the rank with an empty shard has nothing to compare
     results[rank] = dict(
         out=rel(out_r.numpy(), o_ref[:, qlo:qhi]), lse=rel(lse_r.numpy(), l_ref[:, :, qlo:qhi]),
         dq=rel(dq_r.double().numpy(), dq_ref[:, qlo:qhi]),
@@ -127,7 +132,7 @@ def _worker(rank, world, port, causal, results):
     dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("world", [2, 3, 4])
 @pytest.mark.parametrize("causal", [True, False])
 def test_ring_forward_and_backward_match_attention(world, causal):
     port = _free_port()
