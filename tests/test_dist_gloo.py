@@ -40,7 +40,7 @@ def _worker(rank, world, port, results):
 def test_max_over_ranks_with_two_gloo_ranks():
     world = 2
     port = _free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         results = m.dict()
         mp.spawn(_worker, args=(world, port, results), nprocs=world, join=True)
         assert dict(results) == {0: 15.0, 1: 15.0}

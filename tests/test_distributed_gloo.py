@@ -81,7 +81,7 @@ def _worker(rank, world, port, n_local, results):
 @pytest.mark.parametrize("world,n_local", [(2, 1), (3, 2)])
 def test_gathered_shard_partials_merge_to_attention(world, n_local):
     port = _free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         results = m.dict()
         mp.spawn(_worker, args=(world, port, n_local, results), nprocs=world, join=True)
         res = dict(results)
@@ -141,7 +141,7 @@ def _ring_worker(rank, world, port, results):
 @pytest.mark.parametrize("world", [2, 3, 4])
 def test_ring_form_query_blocks_travel_and_partials_merge_at_their_owner(world):
     port = _free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         results = m.dict()
         mp.spawn(_ring_worker, args=(world, port, results), nprocs=world, join=True)
         res = dict(results)

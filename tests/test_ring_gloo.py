@@ -136,7 +136,7 @@ def _worker(rank, world, port, causal, results):
 @pytest.mark.parametrize("causal", [True, False])
 def test_ring_forward_and_backward_match_attention(world, causal):
     port = _free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         results = m.dict()
         mp.spawn(_worker, args=(world, port, causal, results), nprocs=world, join=True)
         res = dict(results)
