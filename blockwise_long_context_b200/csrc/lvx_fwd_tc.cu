@@ -19,8 +19,9 @@
 //               row reads S from TMEM, writes P (bf16) back over S, rescales O
 //               when needed, and finally normalises O and writes the partial.
 // TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,256+D), O_1 [256+D,256+2D).
-// A new S_t is only issued after the previous P_t V MMA completed (P_t lives
-// in S_t's columns), and O_t is only rescaled between two P_t V MMAs.
+// A new S_t is issued only after the P_t V MMA that reads P_t from S_t's
+// columns (the MMAs of one thread execute in issue order, so that read comes
+// first), and O_t is only rescaled between two P_t V MMAs.
 #include "lvx_ptx.cuh"
 #include "lvx_tc.cuh"
 
