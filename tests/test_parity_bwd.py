@@ -111,6 +111,9 @@ def test_backward_far_below_the_maximum():
 
 @pytest.mark.parametrize("cfg", ["C2", "C4", "C3"])
 def test_backward_full_size_sampled(cfg):
+    """dQ on 256 sampled rows of every head and batch (first, last and block-edge
+    rows included); dK, dV on 1024 sampled keys of every KV head of batch 0
+    (C3: its tail keys, see below); the gradient invariants over everything."""
     w = inputs.WORKLOADS[cfg]
     host = inputs.make(w, tensors=("q", "k", "v", "do"))
     out, lse, dq, dk, dv = _run(w, host)
@@ -118,20 +121,39 @@ def test_backward_full_size_sampled(cfg):
         assert torch.isfinite(t.float()).all()
     q, k, v, do = (host[t].double().numpy() for t in ("q", "k", "v", "do"))
     # dQ on sampled rows of every head: needs only those rows' softmax
-    rows = sample_rows(w.S_Q, w.n_blocks, count=96 if cfg == "C3" else 128)
+    rows = sample_rows(w.S_Q, w.n_blocks, count=256)
+    dq_ref = oracle.attention_bwd_rows(q, k, v, do, rows, causal=w.causal)
+    compare(dq[:, rows], dq_ref, "bf16", f"{cfg}: dQ (sampled rows)")
     B0 = 0
-    dq_ref = oracle.attention_bwd_rows(q, k, v, do, rows, causal=w.causal, batches=[B0])[0]
-    compare(dq[B0, rows], dq_ref, "bf16", f"{cfg}: dQ (sampled rows)")
-    # dK, dV on sampled keys of KV head 0, summed over all query rows of its group
     if cfg == "C3":
-        # causal tail keys j >= S-256 get gradient only from rows r >= S-256
+        # causal tail keys j >= S-256 get gradient only from rows r >= S-256 (all
+        # keys of a scaled-down C3 are compared in test_backward_c3_scaled_down)
         keys = np.arange(w.S_KV - 256, w.S_KV)
-        dk_r, dv_r = oracle.attention_bwd_keys(q, k, v, do, keys, [0], causal=True, batches=[B0],
+        heads = list(range(w.H_kv))
+        dk_r, dv_r = oracle.attention_bwd_keys(q, k, v, do, keys, heads, causal=True, batches=[B0],
                                                rows=np.arange(w.S_Q - 256, w.S_Q))
     else:
-        keys = sample_rows(w.S_KV, w.n_blocks, count=384, seed=1)
-        dk_r, dv_r = oracle.attention_bwd_keys(q, k, v, do, keys, [0], causal=w.causal,
+        keys = sample_rows(w.S_KV, w.n_blocks, count=1056, seed=1)   # >= 1024 after the union
+        heads = list(range(w.H_kv))
+        dk_r, dv_r = oracle.attention_bwd_keys(q, k, v, do, keys, heads, causal=w.causal,
                                                batches=[B0])
-    compare(dk[B0, keys, 0], dk_r[0, :, 0], "bf16", f"{cfg}: dK (sampled keys)")
-    compare(dv[B0, keys, 0], dv_r[0, :, 0], "bf16", f"{cfg}: dV (sampled keys)")
+    compare(dk[B0][keys][:, heads], dk_r[0], "bf16", f"{cfg}: dK (sampled keys, every KV head)")
+    compare(dv[B0][keys][:, heads], dv_r[0], "bf16", f"{cfg}: dV (sampled keys, every KV head)")
+    _invariants(w, host, dk, dv)
+
+
+def test_backward_c3_scaled_down():
+    """C3's shape (H = 32, d = 128, n = 8, causal) at S = 16384 on the GPU, with
+    dQ, dK and dV compared in full: every row, key and head (the fp64 oracle
+    evaluates one head at a time, a few seconds each), plus the gradient
+    invariants."""
+    w = inputs.WORKLOADS["C3"].scaled(S_Q=16384, S_KV=16384)
+    host = inputs.make(w, tensors=("q", "k", "v", "do"))
+    out, lse, dq, dk, dv = _run(w, host)
+    for h in range(w.H):
+        sl = {t: host[t][:, :, h:h + 1].double().numpy() for t in ("q", "k", "v", "do")}
+        dq_r, dk_r, dv_r = oracle.attention_bwd(sl["q"], sl["k"], sl["v"], sl["do"], causal=True)
+        compare(dq[:, :, h:h + 1], dq_r, "bf16", f"C3 at S=16384, head {h}: dQ")
+        compare(dk[:, :, h:h + 1], dk_r, "bf16", f"C3 at S=16384, head {h}: dK")
+        compare(dv[:, :, h:h + 1], dv_r, "bf16", f"C3 at S=16384, head {h}: dV")
     _invariants(w, host, dk, dv)
