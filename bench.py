@@ -492,60 +492,67 @@ def run_gpu(a):
 def run_ring(a):
     """Ring Attention (pass-KV), the busiest rank of a ``--ring W`` ring on one GPU.
 
-    Rank W-1 under the causal mask (it computes W-1 full blocks and the diagonal;
-    any rank without the mask): its block partials, their merge and its block
-    gradients, with the library's kernels, timed with CUDA events.  ``value`` is
-    that rank's measured TFLOP/s.  ``projection`` divides the whole problem's
-    FLOPs by the busiest rank's time: what W GPUs would reach if the key/value
-    transfers are hidden, which ``comm`` checks against the measured 770 GB/s
-    NVLink peer-copy bandwidth.  Nothing crosses a GPU boundary in this run."""
+    The rank whose chunk pairs hold the most work (with the contiguous layout
+    under the causal mask: rank W-1, which computes W-1 full blocks and the
+    diagonal; with ``--ring-layout zigzag`` every rank does the same work):
+    its chunk-pair partials, their merge and its chunk-pair gradients, with the
+    library's kernels, timed with CUDA events.  ``value`` is that rank's
+    measured TFLOP/s.  ``projection`` divides the whole problem's FLOPs by the
+    busiest rank's time: what W GPUs would reach if the key/value transfers are
+    hidden, which ``comm`` checks against the measured 770 GB/s NVLink
+    peer-copy bandwidth.  Nothing crosses a GPU boundary in this run."""
     import torch
     from blockwise_long_context_b200 import inputs
     from blockwise_long_context_b200 import binding as lvx
-    from blockwise_long_context_b200.ring import (DIAG, SKIP, kernel_block_grad, kernel_merge,
-                                                  kernel_partial, ring_schedule, shard_bounds)
-    W = a.ring
+    from blockwise_long_context_b200.ring import (DIAG, SKIP, chunks_of, kernel_block_grad,
+                                                  kernel_merge, kernel_partial, pair_mode,
+                                                  shard_bounds)
+    W, layout = a.ring, a.ring_layout
     w = inputs.WORKLOADS[a.workload].scaled(backward=True, d_embed=0)
     if a.s_kv:
         w = w.scaled(S_KV=a.s_kv, S_Q=a.s_kv if w.causal else w.S_Q)
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
+    nC = W if layout == "contiguous" else 2 * W
+    qb = [shard_bounds(w.S_Q, nC, c) for c in range(nC)]
+    kb = [shard_bounds(w.S_KV, nC, c) for c in range(nC)]
+    pair_flops = lambda cq, ck, mode: 3.5 * 4.0 * w.B * w.H * w.d * (
+        (qb[cq][1] - qb[cq][0]) * (qb[cq][1] - qb[cq][0] + 1) / 2 if mode == DIAG
+        else (qb[cq][1] - qb[cq][0]) * (kb[ck][1] - kb[ck][0]))
+    sched = {r: [(st, cq, ck, pair_mode(cq, ck, w.causal)) for st in range(W)
+                 for cq in chunks_of(r, W, layout) for ck in chunks_of((r - st) % W, W, layout)]
+             for r in range(W)}
+    work = {r: sum(pair_flops(cq, ck, m) for _, cq, ck, m in sched[r] if m != SKIP) for r in range(W)}
+    r = max(range(W), key=lambda x: work[x])
+    pairs = [(st, cq, ck, m) for st, cq, ck, m in sched[r] if m != SKIP]
     d = inputs.make_device(w, tensors=("q", "k", "v", "do"), device=dev)
-    r = W - 1 if w.causal else 0
-    qlo, qhi = shard_bounds(w.S_Q, W, r)
-    q_r, do_r = d["q"][:, qlo:qhi].contiguous(), d["do"][:, qlo:qhi].contiguous()
-    sched = [ring_schedule(r, W, s_, w.causal) for s_ in range(W)]
-    blocks = {}
-    for src, mode in sched:
-        if mode != SKIP:
-            lo, hi = shard_bounds(w.S_KV, W, src)
-            blocks[src] = (d["k"][:, lo:hi].contiguous(), d["v"][:, lo:hi].contiguous())
+    cut = lambda t, b: t[:, b[0]:b[1]].contiguous()
+    mine = chunks_of(r, W, layout)
+    q_c = {c: cut(d["q"], qb[c]) for c in mine}
+    do_c = {c: cut(d["do"], qb[c]) for c in mine}
+    kv_c = {ck: (cut(d["k"], kb[ck]), cut(d["v"], kb[ck])) for _, _, ck, _ in pairs}
     del d
-    partial, grad, merge = kernel_partial(), kernel_block_grad(), kernel_merge(q_r)
-    B, S_r, H, hd = q_r.shape
-    o_parts = torch.zeros((W, B, H, S_r, hd), dtype=torch.float32, device=dev)
-    l_parts = torch.full((W, B, H, S_r), float("-inf"), dtype=torch.float32, device=dev)
-    dq = torch.zeros(q_r.shape, dtype=torch.float32, device=dev)
-    acc = {src: (torch.zeros(kv[0].shape, dtype=torch.float32, device=dev),
-                 torch.zeros(kv[1].shape, dtype=torch.float32, device=dev)) for src, kv in blocks.items()}
+    partial, grad = kernel_partial(), kernel_block_grad()
+    B, H, hd = w.B, w.H, w.d
+    slots = {c: W * len(mine) for c in mine}
+    o_parts = {c: torch.zeros((slots[c], B, H, q_c[c].shape[1], hd), dtype=torch.float32, device=dev)
+               for c in mine}
+    l_parts = {c: torch.full((slots[c], B, H, q_c[c].shape[1]), float("-inf"), dtype=torch.float32,
+                             device=dev) for c in mine}
+    dq = {c: torch.zeros(q_c[c].shape, dtype=torch.float32, device=dev) for c in mine}
+    acc = {ck: (torch.zeros(kv[0].shape, dtype=torch.float32, device=dev),
+                torch.zeros(kv[1].shape, dtype=torch.float32, device=dev)) for ck, kv in kv_c.items()}
 
     def rank_step():
-        for s_, (src, mode) in enumerate(sched):
-            if mode != SKIP:
-                partial(q_r, *blocks[src], o_parts[s_:s_ + 1], l_parts[s_:s_ + 1], mode == DIAG)
-        out, lse = merge(o_parts, l_parts)
-        for src, mode in sched:
-            if mode != SKIP:
-                gq, gk, gv = grad(q_r, *blocks[src], out, lse, do_r, mode == DIAG)
-                dq.add_(gq); acc[src][0].add_(gk); acc[src][1].add_(gv)
+        for st, cq, ck, m in pairs:
+            slot = st * len(mine) + chunks_of((r - st) % W, W, layout).index(ck)
+            partial(q_c[cq], *kv_c[ck], o_parts[cq][slot:slot + 1], l_parts[cq][slot:slot + 1],
+                    m == DIAG)
+        merged = {c: kernel_merge(q_c[c])(o_parts[c], l_parts[c]) for c in mine}
+        for st, cq, ck, m in pairs:
+            grad(q_c[cq], *kv_c[ck], merged[cq][0], merged[cq][1], do_c[cq], m == DIAG,
+                 dq[cq], acc[ck][0], acc[ck][1])
 
-    rank_flops = 0.0
-    for src, mode in sched:
-        if mode == SKIP:
-            continue
-        S_k = blocks[src][0].shape[1]
-        pairs = S_r * (S_r + 1) / 2 if mode == DIAG else S_r * S_k
-        rank_flops += 3.5 * 4.0 * B * H * pairs * hd
     for _ in range(max(a.warmup, 3)):
         rank_step()
     torch.cuda.synchronize()
@@ -566,18 +573,19 @@ def run_ring(a):
     kv_step_bytes = 2 * B * (w.S_KV // W) * w.H_kv * w.d * 2
     line = {
         "metric": f"Ring Attention fwd+bwd, busiest rank of a {W}-rank ring, on one GPU",
-        "value": rank_flops / ms / 1e9, "unit": "TFLOP/s", "n_gpus": 1, "steps": a.steps,
+        "value": work[r] / ms / 1e9, "unit": "TFLOP/s", "n_gpus": 1, "steps": a.steps,
         "warmup": max(a.warmup, 3), "ms_per_rank_step": ms, "higher_is_better": True,
         "dtype": "bf16", "data": "synthetic (seeded Gaussian)",
-        "config": {"workload": f"{w.name}: ring of {W} ranks, rank {r} (the busiest)", "B": w.B,
-                   "H": w.H, "H_kv": w.H_kv, "d": w.d, "S_Q": w.S_Q, "S_KV": w.S_KV,
-                   "causal": w.causal, "blocks_computed": sum(m != SKIP for _, m in sched)},
-        "rank_flops": rank_flops,
+        "config": {"workload": f"{w.name}: ring of {W} ranks, {layout} layout, rank {r} (the busiest)",
+                   "B": w.B, "H": w.H, "H_kv": w.H_kv, "d": w.d, "S_Q": w.S_Q, "S_KV": w.S_KV,
+                   "causal": w.causal, "chunk_pairs_computed": len(pairs),
+                   "work_balance": min(work.values()) / work[r]},
+        "rank_flops": work[r],
         "projection": {"ring_tflops": total / ms / 1e9, "per_gpu_tflops": total / ms / 1e9 / W,
                        "assumes": f"{W} GPUs, key/value transfers hidden behind the compute"},
         "comm": {"kv_bytes_per_step": kv_step_bytes,
                  "ms_per_step_at_770_GBps": kv_step_bytes / 770e9 * 1e3,
-                 "compute_ms_per_step": ms / sum(m != SKIP for _, m in sched)},
+                 "compute_ms_per_step": ms / W},
         "clocks": clk,
     }
     print(json.dumps(line), flush=True)
@@ -597,6 +605,8 @@ def main():
                     help="override S_KV (smaller case of the same workload, for profiler captures)")
     ap.add_argument("--ring", type=int, default=0,
                     help="time the busiest rank of a Ring Attention ring of this many ranks (one GPU)")
+    ap.add_argument("--ring-layout", default="contiguous", choices=["contiguous", "zigzag"],
+                    help="rows per rank: one contiguous shard, or chunks r and 2W-1-r of 2W")
     a = ap.parse_args()
     if a.impl == "reference":
         run_reference(a)

@@ -43,6 +43,8 @@ _SIGS = {
     "lvx_attn_fwd_noalloc": ([_vp] * 5 + [_c_int] * 8 + [_c_int, _c_float, _vp], _c_int),
     "lvx_attn_bwd_workspace": ([_c_int] * 7 + [_c_int], _c_size),
     "lvx_attn_bwd": ([_vp] * 9 + [_c_int] * 7 + [_c_int, _c_float, _vp, _c_size, _vp], _c_int),
+    "lvx_attn_bwd_accumulate": ([_vp] * 9 + [_c_int] * 7 + [_c_int, _c_float, _vp, _c_size, _vp],
+                                _c_int),
     "lvx_kv_recompute": ([_vp] * 5 + [_c_int] * 5 + [_c_int, _vp], _c_int),
     "lvx_kv_recompute_bwd": ([_vp] * 8 + [_c_int] * 5 + [_c_int, _vp], _c_int),
     "lvx_last_device_error": ([_vp], _c_int),
@@ -156,6 +158,25 @@ def lvx_attn_bwd(q, k, v, out, lse, dout, dq, dk, dv, causal: bool = False, scal
                               _ptr(dq), _ptr(dk), _ptr(dv), B, H, H_kv, S_Q, S_KV, d,
                               int(causal), _dt(q), float(scale), _ptr(workspace), ws,
                               _stream(stream)), "lvx_attn_bwd")
+
+
+def lvx_attn_bwd_accumulate(q, k, v, out, lse, dout, dq, dk, dv, causal: bool = False,
+                            scale: float = 0.0, workspace: Optional[torch.Tensor] = None,
+                            stream=None) -> None:
+    """As lvx_attn_bwd, with dq, dk, dv float32 arrays the gradients are added to."""
+    B, S_Q, H, d = q.shape
+    S_KV, H_kv = k.shape[1], k.shape[2]
+    for t in (dq, dk, dv):
+        if t.dtype != torch.float32:
+            raise TypeError("lvx_attn_bwd_accumulate adds into float32 gradients")
+    if workspace is None:
+        workspace = bwd_workspace(q, k, causal)
+    ws = workspace.numel() * workspace.element_size()
+    _check(lib().lvx_attn_bwd_accumulate(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse),
+                                         _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), B, H, H_kv, S_Q,
+                                         S_KV, d, int(causal), _dt(q), float(scale),
+                                         _ptr(workspace), ws, _stream(stream)),
+           "lvx_attn_bwd_accumulate")
 
 
 def lvx_kv_recompute(y, w_k, w_v, k, v, H_kv: int, d: int, stream=None) -> None:

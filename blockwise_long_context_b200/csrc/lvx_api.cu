@@ -160,11 +160,15 @@ size_t lvx_attn_bwd_workspace(int B, int H, int H_kv, int S_Q, int S_KV, int d, 
          align256((size_t)B * S_Q * H * d * sizeof(float));
 }
 
-lvx_status lvx_attn_bwd(const void* q, const void* k, const void* v, const void* out,
-                        const float* lse, const void* dout, void* dq, void* dk, void* dv,
-                        int B, int H, int H_kv, int S_Q, int S_KV, int d, int causal,
-                        lvx_dtype dt, float scale, void* workspace, size_t ws_bytes,
-                        lvx_stream stream) {
+namespace {
+
+// The backward with its gradients written (accum = false: dq, dk, dv in dtype
+// dt) or added to float32 arrays (accum = true).
+lvx_status attn_bwd(const void* q, const void* k, const void* v, const void* out,
+                    const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
+                    int H, int H_kv, int S_Q, int S_KV, int d, int causal, lvx_dtype dt,
+                    float scale, void* workspace, size_t ws_bytes, bool accum,
+                    lvx_stream stream) {
   lvx_status st = check_shapes(B, H, H_kv, S_Q, S_KV, d, 1, causal, dt);
   if (st != LVX_OK) return st;
   const void* ptrs[] = {q, k, v, out, lse, dout, dq, dk, dv, workspace};
@@ -182,11 +186,32 @@ lvx_status lvx_attn_bwd(const void* q, const void* k, const void* v, const void*
   cudaError_t e = launch_bwd_pre(out, dout, lse, ND, nlse2, dq_acc, B, H, S_Q, d, dt, s);
   if (e != cudaSuccess) return LVX_ERR_CUDA;
   if (dt == LVX_BF16 && tc_bwd_supported(p))
-    e = launch_bwd_tc(p, q, k, v, dout, nlse2, ND, dq_acc, dk, dv, s);
+    e = launch_bwd_tc(p, q, k, v, dout, nlse2, ND, dq_acc, dk, dv, accum, s);
   else
-    e = launch_bwd_simt(p, dt, q, k, v, dout, lse, ND, dq_acc, dk, dv, s);
+    e = launch_bwd_simt(p, dt, q, k, v, dout, lse, ND, dq_acc, dk, dv, accum, s);
   if (e != cudaSuccess) return LVX_ERR_CUDA;
-  return from_cuda(launch_dq_finalize(dq_acc, dq, (size_t)B * S_Q * H * d, p.scale, dt, s));
+  return from_cuda(
+      launch_dq_finalize(dq_acc, dq, (size_t)B * S_Q * H * d, p.scale, dt, accum, s));
+}
+
+}  // namespace
+
+lvx_status lvx_attn_bwd(const void* q, const void* k, const void* v, const void* out,
+                        const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                        int B, int H, int H_kv, int S_Q, int S_KV, int d, int causal,
+                        lvx_dtype dt, float scale, void* workspace, size_t ws_bytes,
+                        lvx_stream stream) {
+  return attn_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, H, H_kv, S_Q, S_KV, d, causal, dt, scale,
+                  workspace, ws_bytes, false, stream);
+}
+
+lvx_status lvx_attn_bwd_accumulate(const void* q, const void* k, const void* v, const void* out,
+                                   const float* lse, const void* dout, float* dq, float* dk,
+                                   float* dv, int B, int H, int H_kv, int S_Q, int S_KV, int d,
+                                   int causal, lvx_dtype dt, float scale, void* workspace,
+                                   size_t ws_bytes, lvx_stream stream) {
+  return attn_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, H, H_kv, S_Q, S_KV, d, causal, dt, scale,
+                  workspace, ws_bytes, true, stream);
 }
 
 lvx_status lvx_kv_recompute(const void* y, const void* w_k, const void* w_v, void* k, void* v,

@@ -116,7 +116,8 @@ __device__ __forceinline__ int serpentine(int r, int c, int step) {
   return r * step + ((r & 1) ? step - 1 - c : c);
 }
 
-template <int D>
+// ACC: dK, dV added to float32 arrays (map_dk / map_dv are float32 32x32 pieces)
+template <int D, bool ACC>
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
               const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_do,
@@ -542,11 +543,22 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
         ptx::tc_fence_after();
       }
       constexpr int HALF = D / 2;
+      // With ACC, dV and dK are instead added to the caller's float32
+      // arrays with TMA reduce-add, 32 keys x 32 columns at a time: each warp
+      // stages in the 4 KiB of the dS buffer that holds its own dS rows (its
+      // keys' rows of its query half), so it waits only for its own copies, and
+      // before its next dS store.  A key tile no query tile sees adds nothing.
+      // (the base is made opaque here so that these addresses are not hoisted
+      // into the tile loop above, where registers are short)
+      uint8_t* ebase = smem;
+      asm volatile("" : "+l"(ebase));
+      constexpr bool acc = ACC;
+      uint8_t* region = ebase + L::OFF_DS + hf * CHUNK + quarter * 4096;
 #pragma unroll 1
-      for (int which = 0; which < 2; ++which, ++er) {
+      for (int which = 0; which < 2 && !(acc && w.I == 0); ++which) {
         const uint32_t tacc = (which == 0 ? tdV : tdK) + lane_off + HALF * hf;
         const float mul = which == 0 ? 1.f : p.scale;
-        uint8_t* stg = smem + L::OFF_DS + j * 128;
+        uint8_t* stg = ebase + L::OFF_DS + j * 128;
 #pragma unroll 1
         for (int c = 0; c < HALF / 32; ++c) {
           uint32_t r[32];
@@ -556,6 +568,25 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
           } else {
 #pragma unroll
             for (int e = 0; e < 32; ++e) r[e] = 0u;
+          }
+          if constexpr (acc) {
+            if (lane == 0 && (which | c) != 0) bulk_wait_read();   // previous piece read
+            __syncwarp();
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              *reinterpret_cast<uint4*>(region + lane * 128 + ((q ^ (lane & 7)) << 4)) =
+                  make_uint4(__float_as_uint(__uint_as_float(r[4 * q]) * mul),
+                             __float_as_uint(__uint_as_float(r[4 * q + 1]) * mul),
+                             __float_as_uint(__uint_as_float(r[4 * q + 2]) * mul),
+                             __float_as_uint(__uint_as_float(r[4 * q + 3]) * mul));
+            ptx::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_reduce_add_4d(which == 0 ? &map_dv : &map_dk, region, HALF * hf + 32 * c, w.g,
+                                w.n0 + quarter * 32, w.b);
+              bulk_commit();
+            }
+            continue;
           }
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -568,11 +599,13 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
             *reinterpret_cast<uint4*>(stg + (col >> 6) * CHUNK + ((((col & 63) >> 3) ^ (j & 7)) << 4)) = u;
           }
         }
+        if constexpr (acc) continue;
+        ++er;
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
         ptx::mbar_arrive(epi_full);
         if (warp == 4 && lane == 0) {
-          ok = ptx::mbar_wait(epi_full, er & 1, a.err, kErrTimeoutEpilogue, abort_flag);
+          ok = ptx::mbar_wait(epi_full, (er - 1) & 1, a.err, kErrTimeoutEpilogue, abort_flag);
           if (ok) {
             for (int c = 0; c < D / 64; ++c)
               tma_store_4d(which == 0 ? &map_dv : &map_dk, smem + L::OFF_DS + c * CHUNK, 64 * c, w.g,
@@ -582,13 +615,18 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
           }
           ptx::mbar_arrive(epi_free);
         }
-        ok = ptx::mbar_wait(epi_free, er & 1, a.err, kErrTimeoutEpilogue, abort_flag);
+        ok = ptx::mbar_wait(epi_free, (er - 1) & 1, a.err, kErrTimeoutEpilogue, abort_flag);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
       }
+      if (acc && w.I > 0) {
+        if (lane == 0) bulk_wait_read();   // the region takes this warp's next dS rows
+        __syncwarp();
+        ptx::tc_fence_before();
+      }
       if (!ok) break;
     }
-    if (warp == 4 && lane == 0) bulk_wait_all();
+    if ((warp == 4 || ACC) && lane == 0) bulk_wait_all();
   } else {
     ptx::setmaxnreg_dec<kRegsDrain>();
     // ------------------------------------------------------------------ dQ drain
@@ -671,7 +709,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
 template <int D>
 cudaError_t launch(const Problem& p, const void* q, const void* k, const void* v,
                    const void* dout, const float* lse, const float* Dv, float* dq_acc, void* dk,
-                   void* dv, cudaStream_t s) {
+                   void* dv, bool accum, cudaStream_t s) {
   using L = BwdLayout<D>;
   CUtensorMap mq, mk, mv, mdo, mlse, mdd, mdq, mdk, mdv;
   {
@@ -699,12 +737,24 @@ cudaError_t launch(const Problem& p, const void* q, const void* k, const void* v
     if (!encode_tensor_map(&mk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, k, dims, str, box,
                            CU_TENSOR_MAP_SWIZZLE_128B) ||
         !encode_tensor_map(&mv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, v, dims, str, box,
-                           CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_tensor_map(&mdk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, dk, dims, str, box,
-                           CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_tensor_map(&mdv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, dv, dims, str, box,
                            CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
+    if (accum) {
+      // float32 dK, dV, reduced 32 keys x 32 columns at a time
+      const uint64_t str4[3] = {(uint64_t)D * 4, (uint64_t)p.H_kv * D * 4,
+                                (uint64_t)p.S_KV * p.H_kv * D * 4};
+      const uint32_t box4[4] = {32, 1, 32, 1};
+      if (!encode_tensor_map(&mdk, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dk, dims, str4, box4,
+                             CU_TENSOR_MAP_SWIZZLE_128B) ||
+          !encode_tensor_map(&mdv, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dv, dims, str4, box4,
+                             CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    } else if (!encode_tensor_map(&mdk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, dk, dims, str, box,
+                                  CU_TENSOR_MAP_SWIZZLE_128B) ||
+               !encode_tensor_map(&mdv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, dv, dims, str, box,
+                                  CU_TENSOR_MAP_SWIZZLE_128B)) {
+      return cudaErrorInvalidValue;
+    }
   }
   {
     // LSE and D: [B*H, S_Q] fp32 rows; S_Q * 4 bytes must be a multiple of 16
@@ -740,10 +790,10 @@ cudaError_t launch(const Problem& p, const void* q, const void* k, const void* v
     if (ea != cudaSuccess) return ea;
     if (items > n_sm) grid = n_sm;
   }
-  cudaError_t e = cudaFuncSetAttribute(bwd_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       L::BYTES);
+  auto kernel = accum ? bwd_tc_kernel<D, true> : bwd_tc_kernel<D, false>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES);
   if (e != cudaSuccess) return e;
-  bwd_tc_kernel<D><<<(unsigned)grid, kThreads, L::BYTES, s>>>(mq, mk, mv, mdo, mlse, mdd, mdq, mdk, mdv, a);
+  kernel<<<(unsigned)grid, kThreads, L::BYTES, s>>>(mq, mk, mv, mdo, mlse, mdd, mdq, mdk, mdv, a);
   return cudaGetLastError();
 }
 
@@ -754,9 +804,9 @@ bool tc_bwd_supported(const Problem& p) { return (p.d == 64 || p.d == 128) && p.
 
 cudaError_t launch_bwd_tc(const Problem& p, const void* q, const void* k, const void* v,
                           const void* dout, const float* nlse2, const float* nd, float* dq_acc,
-                          void* dk, void* dv, cudaStream_t s) {
-  if (p.d == 128) return launch<128>(p, q, k, v, dout, nlse2, nd, dq_acc, dk, dv, s);
-  if (p.d == 64) return launch<64>(p, q, k, v, dout, nlse2, nd, dq_acc, dk, dv, s);
+                          void* dk, void* dv, bool accum, cudaStream_t s) {
+  if (p.d == 128) return launch<128>(p, q, k, v, dout, nlse2, nd, dq_acc, dk, dv, accum, s);
+  if (p.d == 64) return launch<64>(p, q, k, v, dout, nlse2, nd, dq_acc, dk, dv, accum, s);
   return cudaErrorInvalidValue;
 }
 

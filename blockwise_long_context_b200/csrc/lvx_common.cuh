@@ -65,11 +65,13 @@ cudaError_t launch_merge(const float* o_parts, const float* l_parts, void* out, 
 cudaError_t launch_bwd_pre(const void* out, const void* dout, const float* lse, float* ND,
                            float* nlse2, float* dq_acc, int B, int H, int S_Q, int d, lvx_dtype dt,
                            cudaStream_t s);
+// accum: dk, dv are float32 arrays the gradients are added to
 cudaError_t launch_bwd_simt(const Problem& p, lvx_dtype dt, const void* q, const void* k,
                             const void* v, const void* dout, const float* lse, const float* ND,
-                            float* dq_acc, void* dk, void* dv, cudaStream_t s);
+                            float* dq_acc, void* dk, void* dv, bool accum, cudaStream_t s);
+// dq = scale * dq_acc in dtype dt, or with accum dq (float32) += scale * dq_acc
 cudaError_t launch_dq_finalize(const float* dq_acc, void* dq, size_t count, float scale,
-                               lvx_dtype dt, cudaStream_t s);
+                               lvx_dtype dt, bool accum, cudaStream_t s);
 // C [M][N] row-major = sum over `segments` (1 or 2) of A_g B_g, where element
 // (m, k) of A_g is A[g][m*sam + k*sak] and element (k, n) of B_g is
 // B[g][k*sbk + n*sbn]; every segment has the same K.

@@ -147,15 +147,23 @@ bwd_pre_kernel(const T* __restrict__ out, const T* __restrict__ dout, const floa
   }
 }
 
-template <typename T>
+// ACC: dq (float32) += scale * acc; otherwise dq = scale * acc in T.
+template <typename T, bool ACC>
 __global__ void __launch_bounds__(256)
 dq_finalize_kernel(const float* __restrict__ acc, T* __restrict__ dq, size_t count8, float scale) {
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < count8;
        i += (size_t)gridDim.x * blockDim.x) {
     float x[8];
     Load8<float>::run(acc + i * 8, x);
+    if constexpr (ACC) {
+      float y[8];
+      Load8<float>::run(reinterpret_cast<const float*>(dq) + i * 8, y);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) x[e] *= scale;
+      for (int e = 0; e < 8; ++e) x[e] = fmaf(x[e], scale, y[e]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) x[e] *= scale;
+    }
     Store8<T>::run(dq + i * 8, x);
   }
 }
@@ -201,13 +209,16 @@ cudaError_t launch_bwd_pre(const void* out, const void* dout, const float* lse, 
 }
 
 cudaError_t launch_dq_finalize(const float* dq_acc, void* dq, size_t count, float scale,
-                               lvx_dtype dt, cudaStream_t s) {
+                               lvx_dtype dt, bool accum, cudaStream_t s) {
   const size_t count8 = count / 8;
   const int grid = grid_for(count8, 256);
-  if (dt == LVX_FP32)
-    dq_finalize_kernel<float><<<grid, 256, 0, s>>>(dq_acc, (float*)dq, count8, scale);
+  if (accum)
+    dq_finalize_kernel<float, true><<<grid, 256, 0, s>>>(dq_acc, (float*)dq, count8, scale);
+  else if (dt == LVX_FP32)
+    dq_finalize_kernel<float, false><<<grid, 256, 0, s>>>(dq_acc, (float*)dq, count8, scale);
   else
-    dq_finalize_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(dq_acc, (__nv_bfloat16*)dq, count8, scale);
+    dq_finalize_kernel<__nv_bfloat16, false><<<grid, 256, 0, s>>>(dq_acc, (__nv_bfloat16*)dq,
+                                                                 count8, scale);
   return cudaGetLastError();
 }
 

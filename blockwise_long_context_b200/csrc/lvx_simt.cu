@@ -139,12 +139,13 @@ constexpr int kBwdWarps = 2;
 constexpr int kBwdKeysPerWarp = 16;
 constexpr int kBwdKeys = kBwdWarps * kBwdKeysPerWarp;
 
-template <typename T>
+// TO is the dK / dV element type: T, written; or float with ACC, added to.
+template <typename T, typename TO, bool ACC>
 __global__ void __launch_bounds__(128)
 bwd_simt_kernel(Problem p, const T* __restrict__ q, const T* __restrict__ k,
                 const T* __restrict__ v, const T* __restrict__ dout,
                 const float* __restrict__ lse, const float* __restrict__ ND,
-                float* __restrict__ dq_acc, T* __restrict__ dk, T* __restrict__ dv) {
+                float* __restrict__ dq_acc, TO* __restrict__ dk, TO* __restrict__ dv) {
   __shared__ float ks[kBwdKeys][kMaxD];
   __shared__ float vs[kBwdKeys][kMaxD];
   const int d = p.d;
@@ -231,8 +232,13 @@ bwd_simt_kernel(Problem p, const T* __restrict__ q, const T* __restrict__ k,
     for (int t = 0; t < 4; ++t) {
       const int c = lane + 32 * t;
       if (c < d) {
-        dk[off + c] = Elem<T>::from_f(dk_acc[jj][t] * p.scale);
-        dv[off + c] = Elem<T>::from_f(dv_acc[jj][t]);
+        if constexpr (ACC) {
+          dk[off + c] += dk_acc[jj][t] * p.scale;
+          dv[off + c] += dv_acc[jj][t];
+        } else {
+          dk[off + c] = Elem<T>::from_f(dk_acc[jj][t] * p.scale);
+          dv[off + c] = Elem<T>::from_f(dv_acc[jj][t]);
+        }
       }
     }
   }
@@ -310,16 +316,28 @@ cudaError_t launch_fwd_simt(const Problem& p, lvx_dtype dt, const void* q, const
 
 cudaError_t launch_bwd_simt(const Problem& p, lvx_dtype dt, const void* q, const void* k,
                             const void* v, const void* dout, const float* lse, const float* ND,
-                            float* dq_acc, void* dk, void* dv, cudaStream_t s) {
+                            float* dq_acc, void* dk, void* dv, bool accum, cudaStream_t s) {
   dim3 grid((p.S_KV + kBwdKeys - 1) / kBwdKeys, p.B * p.H_kv);
-  if (dt == LVX_FP32)
-    bwd_simt_kernel<float><<<grid, 32 * kBwdWarps, 0, s>>>(p, (const float*)q, (const float*)k,
-                                                (const float*)v, (const float*)dout, lse, ND,
-                                                dq_acc, (float*)dk, (float*)dv);
-  else
-    bwd_simt_kernel<__nv_bfloat16><<<grid, 32 * kBwdWarps, 0, s>>>(
-        p, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
-        (const __nv_bfloat16*)dout, lse, ND, dq_acc, (__nv_bfloat16*)dk, (__nv_bfloat16*)dv);
+  using bf = __nv_bfloat16;
+  const unsigned nt = 32 * kBwdWarps;
+  if (dt == LVX_FP32) {
+    const float *qq = (const float*)q, *kk = (const float*)k, *vv = (const float*)v,
+                *dd = (const float*)dout;
+    if (accum)
+      bwd_simt_kernel<float, float, true><<<grid, nt, 0, s>>>(p, qq, kk, vv, dd, lse, ND, dq_acc,
+                                                              (float*)dk, (float*)dv);
+    else
+      bwd_simt_kernel<float, float, false><<<grid, nt, 0, s>>>(p, qq, kk, vv, dd, lse, ND, dq_acc,
+                                                               (float*)dk, (float*)dv);
+  } else {
+    const bf *qq = (const bf*)q, *kk = (const bf*)k, *vv = (const bf*)v, *dd = (const bf*)dout;
+    if (accum)
+      bwd_simt_kernel<bf, float, true><<<grid, nt, 0, s>>>(p, qq, kk, vv, dd, lse, ND, dq_acc,
+                                                           (float*)dk, (float*)dv);
+    else
+      bwd_simt_kernel<bf, bf, false><<<grid, nt, 0, s>>>(p, qq, kk, vv, dd, lse, ND, dq_acc,
+                                                         (bf*)dk, (bf*)dv);
+  }
   return cudaGetLastError();
 }
 

@@ -11,12 +11,13 @@ bool tc_fwd_supported(const Problem& p);
 cudaError_t launch_fwd_tc(const Problem& p, const void* q, const void* k, const void* v,
                           void* out, float* lse, float* o_parts, float* l_parts, cudaStream_t s);
 
-// Backward (dK, dV written; dQ accumulated unscaled into dq_acc).  nlse2 is
-// minus the forward's log-sum-exp times log2(e); nd is minus rowsum(dO o O).
+// Backward (dK, dV written in the input dtype, or with accum added to float32
+// arrays; dQ accumulated unscaled into dq_acc).  nlse2 is minus the forward's
+// log-sum-exp times log2(e); nd is minus rowsum(dO o O).
 bool tc_bwd_supported(const Problem& p);
 cudaError_t launch_bwd_tc(const Problem& p, const void* q, const void* k, const void* v,
                           const void* dout, const float* nlse2, const float* nd, float* dq_acc,
-                          void* dk, void* dv, cudaStream_t s);
+                          void* dk, void* dv, bool accum, cudaStream_t s);
 
 // K = y W_k and V = y W_v in one launch (bf16, fp32 accumulation).
 bool tc_gemm_supported(int M, int K, int N);

@@ -40,8 +40,9 @@ import torch.distributed as dist
 from . import binding as lvx
 from .distributed import shard_bounds
 
-__all__ = ["shard_bounds", "ring_schedule", "RingExchange", "run_ring_forward",
-           "run_ring_backward", "ring_attention_forward", "ring_attention_backward"]
+__all__ = ["shard_bounds", "rank_bounds", "chunks_of", "pair_mode", "ring_schedule",
+           "RingExchange", "run_ring_forward", "run_ring_backward", "ring_attention_forward",
+           "ring_attention_backward"]
 
 FULL, DIAG, SKIP = "full", "diag", "skip"
 
@@ -94,17 +95,18 @@ class RingExchange:
         works = dist.batch_isend_irecv(ops) if ops else []
         return list(recvs), works, sends   # the send buffers stay referenced until finish
 
-    def start(self, tensors: Sequence[torch.Tensor], seq_len: Optional[int] = None):
+    def start(self, tensors: Sequence[torch.Tensor], seq_len=None):
         """Sends ``tensors`` to the next rank; the ones received from the previous
         rank have the same shapes except dimension 1, which is ``seq_len`` (the
-        length of the incoming block)."""
+        length of the incoming block; one length, or one per tensor)."""
         if self.world == 1:
             return list(tensors), []
+        lens = seq_len if isinstance(seq_len, (list, tuple)) else [seq_len] * len(tensors)
         recv = []
-        for t in tensors:
+        for t, n in zip(tensors, lens):
             shape = list(t.shape)
-            if seq_len is not None:
-                shape[1] = seq_len
+            if n is not None:
+                shape[1] = n
             recv.append(torch.empty(shape, dtype=t.dtype, device=t.device))
         return self.exchange(tensors, (self.rank + 1) % self.world, recv,
                              (self.rank - 1) % self.world)
@@ -116,68 +118,148 @@ class RingExchange:
             w.wait()
         return recv
 
-    def pass_on(self, tensors: Sequence[torch.Tensor], seq_len: Optional[int] = None
-                ) -> List[torch.Tensor]:
+    def pass_on(self, tensors: Sequence[torch.Tensor], seq_len=None) -> List[torch.Tensor]:
         return self.finish(self.start(tensors, seq_len))
 
 
 PartialFn = Callable[[torch.Tensor, torch.Tensor, torch.Tensor, torch.Tensor, torch.Tensor, bool], None]
 MergeFn = Callable[[torch.Tensor, torch.Tensor], Tuple[torch.Tensor, torch.Tensor]]
-GradFn = Callable[..., Tuple[torch.Tensor, torch.Tensor, torch.Tensor]]
+GradFn = Callable[..., None]
+
+
+CONTIGUOUS, ZIGZAG = "contiguous", "zigzag"
+
+
+def chunks_of(rank: int, world: int, layout: str = CONTIGUOUS) -> List[int]:
+    """The chunks of the sequence rank ``rank`` holds, in the order it holds them:
+    contiguous, one chunk of W (chunk r); zigzag, two of 2W (chunks r and
+    2W - 1 - r), which gives every rank the same causal work at every step."""
+    if layout == CONTIGUOUS:
+        return [rank]
+    if layout == ZIGZAG:
+        return [rank, 2 * world - 1 - rank]
+    raise ValueError(f"unknown layout {layout!r}")
+
+
+def rank_bounds(S: int, world: int, rank: int, layout: str = CONTIGUOUS) -> List[Tuple[int, int]]:
+    """Rows [lo, hi) of a length-S sequence that rank ``rank`` holds, chunk by
+    chunk; its local tensors are these rows concatenated in this order."""
+    n = world if layout == CONTIGUOUS else 2 * world
+    return [shard_bounds(S, n, c) for c in chunks_of(rank, world, layout)]
+
+
+def pair_mode(cq: int, ck: int, causal: bool) -> str:
+    """Query chunk ``cq`` against key chunk ``ck``: in full, with the diagonal
+    mask, or skipped (every key of a later chunk is masked)."""
+    if not causal or ck < cq:
+        return FULL
+    return DIAG if ck == cq else SKIP
+
+
+class _Chunks:
+    """Chunk lengths of a sequence sharded over the ranks (all ranks agree: the
+    total length comes from the gathered local lengths)."""
+
+    def __init__(self, local_len: int, exchange: "RingExchange", layout: str, device):
+        world = exchange.world
+        self.total = sum(exchange.lengths(local_len, device))
+        self.n = world if layout == CONTIGUOUS else 2 * world
+        self.world, self.layout = world, layout
+
+    def lens(self, rank: int) -> List[int]:
+        return [hi - lo for lo, hi in rank_bounds(self.total, self.world, rank, self.layout)]
+
+
+def _split(t: torch.Tensor, lens: Sequence[int], dim: int = 1) -> List[torch.Tensor]:
+    out, o = [], 0
+    for n in lens:
+        out.append(t.narrow(dim, o, n).contiguous())
+        o += n
+    if o != t.shape[dim]:
+        raise ValueError("local rows do not match the layout's chunks (cut them with rank_bounds)")
+    return out
 
 
 def run_ring_forward(q, k, v, partial_fn: PartialFn, merge_fn: MergeFn, exchange: RingExchange,
-                     causal: bool = False):
-    """q [B, S_r, H, d], k, v [B, S_kv_r, H_kv, d]: this rank's blocks.
-    ``partial_fn(q, k_blk, v_blk, O [1,B,H,S_r,d], L [1,B,H,S_r], diagonal)`` writes
-    one block partial; ``merge_fn(O_parts, L_parts)`` returns (out, lse).  The next
-    block's transfer is started before the current block's partial is computed."""
+                     causal: bool = False, layout: str = CONTIGUOUS):
+    """q [B, S_r, H, d], k, v [B, S_kv_r, H_kv, d]: this rank's rows (its chunks,
+    concatenated).  ``partial_fn(q, k_blk, v_blk, O [1,B,H,S,d], L [1,B,H,S],
+    diagonal)`` writes one chunk pair's partial; ``merge_fn(O_parts, L_parts)``
+    returns (out, lse) for one query chunk.  The next block's transfer is started
+    before the current block's partials are computed."""
     world, rank = exchange.world, exchange.rank
-    B, S_r, H, d = q.shape
-    kv_len = exchange.lengths(k.shape[1], k.device)   # shards may differ in length
-    o_parts = torch.zeros((world, B, H, S_r, d), dtype=torch.float32, device=q.device)
-    l_parts = torch.full((world, B, H, S_r), float("-inf"), dtype=torch.float32, device=q.device)
-    k_cur, v_cur = k, v
+    B, _, H, d = q.shape
+    qc = _Chunks(q.shape[1], exchange, layout, q.device)
+    kc = _Chunks(k.shape[1], exchange, layout, k.device)
+    mine = chunks_of(rank, world, layout)
+    nloc = len(mine)
+    q_ch = _split(q, qc.lens(rank))
+    k_cur, v_cur = _split(k, kc.lens(rank)), _split(v, kc.lens(rank))
+    o_parts = [torch.zeros((world * nloc, B, H, t.shape[1], d), dtype=torch.float32, device=q.device)
+               for t in q_ch]
+    l_parts = [torch.full((world * nloc, B, H, t.shape[1]), float("-inf"), dtype=torch.float32,
+                          device=q.device) for t in q_ch]
     for step in range(world):
-        _, mode = ring_schedule(rank, world, step, causal)
+        theirs = chunks_of((rank - step) % world, world, layout)
         handle = None
         if step + 1 < world:
-            nxt = ring_schedule(rank, world, step + 1, causal)[0]
-            handle = exchange.start([k_cur, v_cur], kv_len[nxt])
-        if mode != SKIP:
-            partial_fn(q, k_cur, v_cur, o_parts[step:step + 1], l_parts[step:step + 1], mode == DIAG)
+            nxt = kc.lens((rank - step - 1) % world)
+            handle = exchange.start(k_cur + v_cur, nxt + nxt)
+        for iq, cq in enumerate(mine):
+            for ik, ck in enumerate(theirs):
+                mode = pair_mode(cq, ck, causal)
+                if mode != SKIP:
+                    slot = step * nloc + ik
+                    partial_fn(q_ch[iq], k_cur[ik], v_cur[ik], o_parts[iq][slot:slot + 1],
+                               l_parts[iq][slot:slot + 1], mode == DIAG)
         if handle is not None:
-            k_cur, v_cur = exchange.finish(handle)
-    return merge_fn(o_parts, l_parts)
+            recv = exchange.finish(handle)
+            k_cur, v_cur = recv[:nloc], recv[nloc:]
+    merged = [merge_fn(o, l) for o, l in zip(o_parts, l_parts)]
+    if nloc == 1:
+        return merged[0]
+    return torch.cat([m[0] for m in merged], dim=1), torch.cat([m[1] for m in merged], dim=2)
 
 
 def run_ring_backward(q, k, v, out, lse, do, grad_fn: GradFn, exchange: RingExchange,
-                      causal: bool = False):
-    """Gradients of this rank's blocks: (dq [B,S_r,H,d], dk, dv [B,S_kv_r,H_kv,d]) in
-    float32.  ``grad_fn(q, k_blk, v_blk, out, lse, do, diagonal)`` returns one block
-    pair's contributions (dq_part, dk_part, dv_part) with the global ``lse``."""
+                      causal: bool = False, layout: str = CONTIGUOUS):
+    """Gradients of this rank's rows: (dq [B,S_r,H,d], dk, dv [B,S_kv_r,H_kv,d]) in
+    float32.  ``grad_fn(q, k_blk, v_blk, out, lse, do, diagonal, dq, dk, dv)`` adds
+    one chunk pair's contributions, computed with the global ``lse``, to the
+    float32 accumulators dq, dk, dv."""
     world, rank = exchange.world, exchange.rank
-    kv_len = exchange.lengths(k.shape[1], k.device)
-    dq = torch.zeros(q.shape, dtype=torch.float32, device=q.device)
-    dk_acc = torch.zeros(k.shape, dtype=torch.float32, device=k.device)
-    dv_acc = torch.zeros(v.shape, dtype=torch.float32, device=v.device)
-    k_cur, v_cur = k, v
+    qc = _Chunks(q.shape[1], exchange, layout, q.device)
+    kc = _Chunks(k.shape[1], exchange, layout, k.device)
+    mine = chunks_of(rank, world, layout)
+    nloc = len(mine)
+    ql = qc.lens(rank)
+    q_ch, out_ch, do_ch = _split(q, ql), _split(out, ql), _split(do, ql)
+    lse_ch = _split(lse, ql, dim=2)
+    k_cur, v_cur = _split(k, kc.lens(rank)), _split(v, kc.lens(rank))
+    f32 = lambda t: torch.zeros(t.shape, dtype=torch.float32, device=t.device)
+    dq = [f32(t) for t in q_ch]
+    dk_acc, dv_acc = [f32(t) for t in k_cur], [f32(t) for t in v_cur]
     for step in range(world):
-        _, mode = ring_schedule(rank, world, step, causal)
+        theirs = chunks_of((rank - step) % world, world, layout)
         # the block (and accumulators) this rank holds next: after the last step,
-        # the accumulators of its own block come home
-        nxt = ring_schedule(rank, world, step + 1, causal)[0] if step + 1 < world else rank
-        handle = exchange.start([k_cur, v_cur], kv_len[nxt]) if step + 1 < world else None
-        if mode != SKIP:
-            dq_p, dk_p, dv_p = grad_fn(q, k_cur, v_cur, out, lse, do, mode == DIAG)
-            dq += dq_p
-            dk_acc += dk_p
-            dv_acc += dv_p
+        # the accumulators of its own chunks come home
+        nxt = kc.lens((rank - step - 1) % world) if step + 1 < world else kc.lens(rank)
+        handle = exchange.start(k_cur + v_cur, nxt + nxt) if step + 1 < world else None
+        for iq, cq in enumerate(mine):
+            for ik, ck in enumerate(theirs):
+                mode = pair_mode(cq, ck, causal)
+                if mode == SKIP:
+                    continue
+                grad_fn(q_ch[iq], k_cur[ik], v_cur[ik], out_ch[iq], lse_ch[iq], do_ch[iq],
+                        mode == DIAG, dq[iq], dk_acc[ik], dv_acc[ik])
         # the accumulators travel with their block; the last pass returns them home
-        dk_acc, dv_acc = exchange.pass_on([dk_acc, dv_acc], kv_len[nxt])
+        recv = exchange.pass_on(dk_acc + dv_acc, nxt + nxt)
+        dk_acc, dv_acc = recv[:nloc], recv[nloc:]
         if handle is not None:
-            k_cur, v_cur = exchange.finish(handle)
-    return dq, dk_acc, dv_acc
+            recv = exchange.finish(handle)
+            k_cur, v_cur = recv[:nloc], recv[nloc:]
+    cat = lambda ts: ts[0] if len(ts) == 1 else torch.cat(ts, dim=1)
+    return cat(dq), cat(dk_acc), cat(dv_acc)
 
 
 def kernel_partial(scale: float = 0.0, stream=None) -> PartialFn:
@@ -198,10 +280,10 @@ def kernel_partial(scale: float = 0.0, stream=None) -> PartialFn:
 
 
 def kernel_merge(like: torch.Tensor, stream=None) -> MergeFn:
-    """The library's merge kernel, output in ``like``'s dtype and shape."""
+    """The library's merge kernel, output in ``like``'s dtype (shape from the partials)."""
     def fn(o_parts, l_parts):
-        B, S_r, H, _ = like.shape
-        out = torch.empty_like(like)
+        _, B, H, S_r, d = o_parts.shape
+        out = torch.empty((B, S_r, H, d), dtype=like.dtype, device=like.device)
         lse = torch.empty(B, H, S_r, dtype=torch.float32, device=like.device)
         if S_r > 0:
             lvx.lvx_merge_partials(o_parts, l_parts, out, lse, stream)
@@ -209,16 +291,16 @@ def kernel_merge(like: torch.Tensor, stream=None) -> MergeFn:
     return fn
 
 
-def kernel_block_grad(scale: float = 0.0) -> GradFn:
+def kernel_block_grad(scale: float = 0.0, stream=None) -> GradFn:
     """One block pair's gradient contributions with the library's fused backward
-    (it recomputes P from the given global log-sum-exp and D from out and do)."""
-    def fn(q, k_blk, v_blk, out, lse, do, diagonal):
+    (it recomputes P from the given global log-sum-exp and D from out and do),
+    added in float32 to the accumulators by the kernels themselves
+    (``lvx_attn_bwd_accumulate``): no part is rounded to the input dtype."""
+    def fn(q, k_blk, v_blk, out, lse, do, diagonal, dq, dk, dv):
         if q.shape[1] == 0 or k_blk.shape[1] == 0:
-            z = lambda t: torch.zeros(t.shape, dtype=torch.float32, device=t.device)
-            return z(q), z(k_blk), z(v_blk)
-        dq, dk, dv = lvx.attention_backward(q, k_blk, v_blk, out, lse, do, causal=diagonal,
-                                            scale=scale)
-        return dq.float(), dk.float(), dv.float()
+            return
+        lvx.lvx_attn_bwd_accumulate(q, k_blk, v_blk, out, lse, do, dq, dk, dv, causal=diagonal,
+                                    scale=scale, stream=stream)
     return fn
 
 
@@ -228,19 +310,21 @@ def _require_cuda(t: torch.Tensor, what: str) -> None:
 
 
 def ring_attention_forward(q, k, v, group=None, causal: bool = False, scale: float = 0.0,
-                           stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+                           stream=None, layout: str = CONTIGUOUS) -> Tuple[torch.Tensor, torch.Tensor]:
     """Attention of this rank's query rows over the key/value sequence sharded
-    across the ranks of ``group`` -> out [B, S_r, H, d], lse [B, H, S_r] float32."""
+    across the ranks of ``group`` (rows cut with ``rank_bounds``) ->
+    out [B, S_r, H, d], lse [B, H, S_r] float32."""
     _require_cuda(q, "ring_attention_forward")
     return run_ring_forward(q, k, v, kernel_partial(scale, stream), kernel_merge(q, stream),
-                            RingExchange(group), causal)
+                            RingExchange(group), causal, layout)
 
 
 def ring_attention_backward(q, k, v, out, lse, do, group=None, causal: bool = False,
-                            scale: float = 0.0) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
-    """dq, dk, dv of this rank's blocks (input dtype), from the ring forward's
+                            scale: float = 0.0, layout: str = CONTIGUOUS
+                            ) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """dq, dk, dv of this rank's rows (input dtype), from the ring forward's
     out and lse."""
     _require_cuda(q, "ring_attention_backward")
     dq, dk, dv = run_ring_backward(q, k, v, out, lse, do, kernel_block_grad(scale),
-                                   RingExchange(group), causal)
+                                   RingExchange(group), causal, layout)
     return dq.to(q.dtype), dk.to(k.dtype), dv.to(v.dtype)

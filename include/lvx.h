@@ -198,6 +198,22 @@ lvx_status lvx_attn_bwd(const void* q, const void* k, const void* v, const void*
                         lvx_stream stream);
 
 /*
+ * The same backward, with the gradients ADDED to caller-owned float32 arrays
+ * instead of written: dq [B, S_Q, H, d], dk, dv [B, S_KV, H_kv, d] float32
+ * (device, 16-byte aligned) receive dq += dQ, dk += dK, dv += dV of this
+ * call.  For gradients summed over several calls -- the key/value blocks of a
+ * ring (Ring Attention with Blockwise Transformers page, abstract) or any
+ * split of the keys -- without rounding each part to the input dtype.  The
+ * caller zeroes the arrays before the first call.  Inputs, workspace, shapes
+ * and errors as lvx_attn_bwd; the calls of one stream accumulate in order.
+ */
+lvx_status lvx_attn_bwd_accumulate(const void* q, const void* k, const void* v, const void* out,
+                                   const float* lse, const void* dout, float* dq, float* dk,
+                                   float* dv, int B, int H, int H_kv, int S_Q, int S_KV, int d,
+                                   int causal, lvx_dtype dt, float scale, void* workspace,
+                                   size_t ws_bytes, lvx_stream stream);
+
+/*
  * Key/value recomputation from the shared visual features.
  *   LV-XAttn review page, "What carries the argument" and Figure 6: one copy
  *   of y serves every cross-attention layer, and K, V are regenerated from it

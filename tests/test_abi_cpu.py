@@ -86,6 +86,14 @@ def test_bwd_and_kv_reject_invalid_arguments():
     assert L.lvx_attn_bwd(*bad) == INVALID
     bad = list(args); bad[14] = 256
     assert L.lvx_attn_bwd(*bad) == UNSUPPORTED
+    # the accumulating form validates the same way
+    assert L.lvx_attn_bwd_accumulate(*args) == WORKSPACE
+    bad = list(args); bad[6] = None                        # dq
+    assert L.lvx_attn_bwd_accumulate(*bad) == INVALID
+    bad = list(args); bad[8] = 24                          # dv misaligned
+    assert L.lvx_attn_bwd_accumulate(*bad) == INVALID
+    bad = list(args); bad[15] = 1; bad[12] = 8             # causal with S_Q != S_KV
+    assert L.lvx_attn_bwd_accumulate(*bad) == UNSUPPORTED
     assert L.lvx_kv_recompute(P16, P16, None, P16, P16, 1, 4, 64, 1, 64, lvx.LVX_BF16, None) == INVALID
     assert L.lvx_kv_recompute(P16, P16, P16, P16, P16, 1, 0, 64, 1, 64, lvx.LVX_BF16, None) == INVALID
     assert L.lvx_kv_recompute(P16, P16, P16, P16, P16, 1, 4, 64, 1, 64, 9, None) == UNSUPPORTED

@@ -157,3 +157,39 @@ def test_backward_c3_scaled_down():
         compare(dk[:, :, h:h + 1], dk_r, "bf16", f"C3 at S=16384, head {h}: dK")
         compare(dv[:, :, h:h + 1], dv_r, "bf16", f"C3 at S=16384, head {h}: dV")
     _invariants(w, host, dk, dv)
+
+
+ACCUM = [
+    # name,                B, H, H_kv, d,  S_Q, S_KV, causal, dtype   (path)
+    ("tc_d128_gqa",         1, 4, 2,  128, 300, 1000, False, "bf16"),  # tensor cores
+    ("tc_causal",           1, 2, 2,  128, 700,  700, True,  "bf16"),
+    ("tc_d64",              2, 2, 1,   64, 256,  777, False, "bf16"),
+    ("simt_rows_not_4k",    1, 2, 1,  128, 130,  513, False, "bf16"),  # S_Q % 4 != 0: CUDA cores
+    ("simt_d96",            1, 2, 1,   96, 100,  300, False, "bf16"),
+    ("simt_f32",            1, 2, 1,   64, 128,  256, False, "f32"),
+]
+
+
+@pytest.mark.parametrize("case", ACCUM, ids=[c[0] for c in ACCUM])
+def test_backward_accumulate_adds_to_float32(case):
+    """lvx_attn_bwd_accumulate adds the gradients to float32 arrays: starting
+    from nonzero arrays A and calling it twice gives A + 2 * gradient."""
+    name, *shape = case
+    w = _workload(*shape)
+    host = inputs.make(w, tensors=("q", "k", "v", "do"))
+    dev = {t: x.cuda() for t, x in host.items()}
+    out, lse = lvx.attention_forward(dev["q"], dev["k"], dev["v"], w.n_blocks, w.causal)
+    g = torch.Generator(device="cuda").manual_seed(3)
+    start = [torch.randn(t.shape, generator=g, device="cuda") for t in (dev["q"], dev["k"], dev["v"])]
+    acc = [t.clone() for t in start]
+    ws = lvx.bwd_workspace(dev["q"], dev["k"], w.causal)
+    for _ in range(2):
+        lvx.lvx_attn_bwd_accumulate(dev["q"], dev["k"], dev["v"], out, lse, dev["do"], *acc,
+                                    causal=w.causal, workspace=ws)
+    lvx.lvx_last_device_error()
+    torch.cuda.synchronize()
+    q, k, v, do = (host[t].double().numpy() for t in ("q", "k", "v", "do"))
+    refs = oracle.attention_bwd(q, k, v, do, causal=w.causal)
+    for nm, a, s0, r in zip(("dQ", "dK", "dV"), acc, start, refs):
+        got = (a - s0).double().cpu().numpy() / 2.0
+        compare(got, r, w.dtype, f"accumulate {name}: {nm}")

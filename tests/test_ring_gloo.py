@@ -46,6 +46,33 @@ def test_schedule_visits_every_block_once(world, causal):
                 ring_schedule((rank - 1) % world, world, s - 1, causal)[0]
 
 
+@pytest.mark.parametrize("world", [2, 3, 4, 8])
+def test_zigzag_balances_causal_work(world):
+    """With the zigzag layout every rank computes the same causal work at every
+    step (two chunk-squares: two full pairs, or one full pair and two diagonal
+    halves); with the contiguous layout the last rank computes W - 1 full blocks
+    and the diagonal while rank 0 computes only its diagonal."""
+    sys.path.insert(0, ROOT)
+    from blockwise_long_context_b200.ring import chunks_of, pair_mode
+    weight = {"full": 1.0, "diag": 0.5, "skip": 0.0}
+    for s in range(world):
+        per_rank = []
+        for r in range(world):
+            theirs = chunks_of((r - s) % world, world, "zigzag")
+            per_rank.append(sum(weight[pair_mode(cq, ck, True)]
+                                for cq in chunks_of(r, world, "zigzag") for ck in theirs))
+        assert per_rank == [2.0] * world, (s, per_rank)
+    totals = [sum(weight[pair_mode(r, (r - s) % world, True)] for s in range(world))
+              for r in range(world)]
+    assert totals == [r + 0.5 for r in range(world)]
+    # the zigzag chunks of all ranks tile the sequence once
+    for S in (9, 23, 64, 1000):
+        from blockwise_long_context_b200.ring import rank_bounds
+        rows = sorted(i for r in range(world) for lo, hi in rank_bounds(S, world, r, "zigzag")
+                      for i in range(lo, hi))
+        assert rows == list(range(S))
+
+
 def _block_grad(q, k, v, out, lse, do, diagonal, scale):
     """Textbook blockwise gradient of one (query block, key block) pair with the
     rows' global log-sum-exp: P = exp(s q.k - lse), dV = P^T dO, dP = dO V^T,
@@ -70,7 +97,12 @@ def _block_grad(q, k, v, out, lse, do, diagonal, scale):
     return dq, dk, dv
 
 
-def _worker(rank, world, port, causal, results):
+def _rows(a, bounds):
+    """This rank's rows: its chunks, concatenated in order."""
+    return np.concatenate([a[:, lo:hi] for lo, hi in bounds], axis=1)
+
+
+def _worker(rank, world, port, causal, layout, results):
     import datetime
     import torch.distributed as dist
     sys.path.insert(0, ROOT)
@@ -78,8 +110,8 @@ def _worker(rank, world, port, causal, results):
     dist.init_process_group("gloo", rank=rank, world_size=world,
                             timeout=datetime.timedelta(seconds=60))
     import oracle
-    from blockwise_long_context_b200.ring import (RingExchange, run_ring_backward,
-                                                  run_ring_forward, shard_bounds)
+    from blockwise_long_context_b200.ring import (RingExchange, rank_bounds, run_ring_backward,
+                                                  run_ring_forward)
     rng = np.random.default_rng(21)                  # the same full problem on every rank
     B, H, H_kv, d = 2, 4, 2, 8
     S_Q, S_KV = (23, 23) if causal else (13, 29)
@@ -90,10 +122,10 @@ def _worker(rank, world, port, causal, results):
     v = rng.standard_normal((B, S_KV, H_kv, d))
     do = rng.standard_normal((B, S_Q, H, d))
     scale = 1.0 / np.sqrt(d)
-    qlo, qhi = shard_bounds(S_Q, world, rank)
-    klo, khi = shard_bounds(S_KV, world, rank)
+    qb, kb = rank_bounds(S_Q, world, rank, layout), rank_bounds(S_KV, world, rank, layout)
     t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).float()
-    q_r, k_r, v_r, do_r = t(q[:, qlo:qhi]), t(k[:, klo:khi]), t(v[:, klo:khi]), t(do[:, qlo:qhi])
+    q_r, do_r = t(_rows(q, qb)), t(_rows(do, qb))
+    k_r, v_r = t(_rows(k, kb)), t(_rows(v, kb))
 
     def partial(qq, kk, vv, o, l, diagonal):
         if qq.shape[1] == 0 or kk.shape[1] == 0:
@@ -109,36 +141,40 @@ def _worker(rank, world, port, causal, results):
         return torch.from_numpy(out), torch.from_numpy(lse)
 
     ex = RingExchange()
-    out_r, lse_r = run_ring_forward(q_r, k_r, v_r, partial, merge, ex, causal)
+    out_r, lse_r = run_ring_forward(q_r, k_r, v_r, partial, merge, ex, causal, layout)
 
-    def grad(qq, kk, vv, oo, ll, dd, diagonal):
-        return tuple(torch.from_numpy(a) for a in _block_grad(
-            qq.double().numpy(), kk.double().numpy(), vv.double().numpy(), oo.double().numpy(),
-            ll.double().numpy(), dd.double().numpy(), diagonal, scale))
+    def grad(qq, kk, vv, oo, ll, dd, diagonal, dq_acc, dk_acc, dv_acc):
+        parts = _block_grad(qq.double().numpy(), kk.double().numpy(), vv.double().numpy(),
+                            oo.double().numpy(), ll.double().numpy(), dd.double().numpy(),
+                            diagonal, scale)
+        for acc, part in zip((dq_acc, dk_acc, dv_acc), parts):
+            acc += torch.from_numpy(part).float()
 
-    dq_r, dk_r, dv_r = run_ring_backward(q_r, k_r, v_r, out_r, lse_r, do_r, grad, ex, causal)
+    dq_r, dk_r, dv_r = run_ring_backward(q_r, k_r, v_r, out_r, lse_r, do_r, grad, ex, causal, layout)
 
     qf, kf, vf, dof = (t(a).double().numpy() for a in (q, k, v, do))   # the float32 inputs
     o_ref, l_ref = oracle.attention_fwd(qf, kf, vf, causal=causal)
     dq_ref, dk_ref, dv_ref = oracle.attention_bwd(qf, kf, vf, dof, causal=causal)
     rel = lambda a, b: (float(np.abs(a - b).max() / max(np.abs(b).max(), 1e-30)) if b.size
                         else 0.0)   # the rank with an empty shard has nothing to compare
+    lse_rows = np.concatenate([l_ref[:, :, lo:hi] for lo, hi in qb], axis=2)
     results[rank] = dict(
-        out=rel(out_r.numpy(), o_ref[:, qlo:qhi]), lse=rel(lse_r.numpy(), l_ref[:, :, qlo:qhi]),
-        dq=rel(dq_r.double().numpy(), dq_ref[:, qlo:qhi]),
-        dk=rel(dk_r.double().numpy(), dk_ref[:, klo:khi]),
-        dv=rel(dv_r.double().numpy(), dv_ref[:, klo:khi]))
+        out=rel(out_r.numpy(), _rows(o_ref, qb)), lse=rel(lse_r.numpy(), lse_rows),
+        dq=rel(dq_r.double().numpy(), _rows(dq_ref, qb)),
+        dk=rel(dk_r.double().numpy(), _rows(dk_ref, kb)),
+        dv=rel(dv_r.double().numpy(), _rows(dv_ref, kb)))
     dist.barrier()
     dist.destroy_process_group()
 
 
 @pytest.mark.parametrize("world", [2, 3, 4])
 @pytest.mark.parametrize("causal", [True, False])
-def test_ring_forward_and_backward_match_attention(world, causal):
+@pytest.mark.parametrize("layout", ["contiguous", "zigzag"])
+def test_ring_forward_and_backward_match_attention(world, causal, layout):
     port = _free_port()
     with mp.get_context("spawn").Manager() as m:
         results = m.dict()
-        mp.spawn(_worker, args=(world, port, causal, results), nprocs=world, join=True)
+        mp.spawn(_worker, args=(world, port, causal, layout, results), nprocs=world, join=True)
         res = dict(results)
     assert sorted(res) == list(range(world))
     for rank, errs in res.items():
