@@ -8,19 +8,26 @@ blockwise attention of its queries against the block it holds while that
 block moves on to the next worker.  The partial outputs are combined by the
 same rescaling as the merge of the block partials.
 
-Layout: rank r of W holds rows ``shard_bounds(S, W, r)`` of Q and of K, V.
+Layouts: the sequence is cut into chunks with ``shard_bounds``.  Contiguous:
+W chunks, rank r holds chunk r.  Zigzag: 2W chunks, rank r holds chunks r and
+2W - 1 - r (its local tensors are the two concatenated; ``rank_bounds``
+gives the rows).  At step s rank r holds the chunks of rank (r - s) mod W.
 For self-attention with the causal mask (the plainest reading, as for the
-single-GPU kernels: key j is visible to query row i iff j <= i), at step s
-rank r holds the block of rank src = (r - s) mod W; the pair is computed in
-full if src < r, with the diagonal mask if src == r, and skipped if src > r
-(its partial is the empty (0, -inf)).  Without the mask every pair is
-computed (cross-attention whose query and key sequences are both sharded).
+single-GPU kernels: key j is visible to query row i iff j <= i), a query
+chunk is computed against an earlier key chunk in full, against its own
+chunk with the diagonal mask, and not against a later one (that partial is
+the empty (0, -inf)).  With the contiguous layout the last rank then does
+W - 1 full blocks and the diagonal while the first does only its diagonal;
+the zigzag layout gives every rank the same work at every step.  Without
+the mask every pair is computed (cross-attention whose query and key
+sequences are both sharded).
 
-Backward: each block's dK, dV accumulators travel with it; a step adds the
-contribution of the local query rows, computed with their global
+Backward: each chunk's dK, dV accumulators (float32) travel with it; a step
+adds the contribution of the local query rows, computed with their global
 log-sum-exp and D = rowsum(dO o O) (the blockwise form of the exact
-gradient).  After W steps and W passes of the accumulators each is back with
-the block's owner.  The pages leave the backward unspecified (LV-XAttn review
+gradient), with ``lvx_attn_bwd_accumulate``, which adds in float32 without
+rounding each part to the input dtype.  After W steps and W passes of the
+accumulators each is back with the chunk's owner.  The pages leave the backward unspecified (LV-XAttn review
 page, referee report, major comment 1); this is the textbook gradient, as in
 the single-GPU backward.
 
