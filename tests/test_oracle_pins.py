@@ -83,6 +83,32 @@ def test_identical_keys_give_mean_of_values():
             np.testing.assert_allclose(lse[b, h], q[b, :, h] @ k[b, 0, g] / math.sqrt(8) + math.log(9), atol=1e-13)
 
 
+def test_dominant_key_far_above_the_rest():
+    """Logits spread over hundreds of natural-log units (the regime the GPU
+    parity cases with rising logits and far-below arguments use): a key whose
+    logit exceeds every other by > 100 returns its value, and the LSE is that
+    logit plus a term below e^-100; two equal spikes return the mean of their
+    values with LSE = spike + ln 2 (closed forms)."""
+    d, S = 8, 40
+    q = np.zeros((1, 1, 1, d)); q[0, 0, 0, 0] = 1.0
+    k = np.zeros((1, S, 1, d)); k[0, :, 0, 0] = np.linspace(-300.0, 0.0, S)
+    v = _rand((1, S, 1, d), 7)
+    sc = 1.0
+    k[0, 17, 0, 0] = 150.0                       # 150 above the next largest logit (0)
+    out, lse = oracle.attention_fwd(q, k, v, scale=sc)
+    assert np.abs(out[0, 0, 0] - v[0, 17, 0]).max() < 1e-60
+    assert abs(lse[0, 0, 0] - 150.0) < 1e-12
+    k[0, 23, 0, 0] = 150.0                       # a second, equal spike
+    out, lse = oracle.attention_fwd(q, k, v, scale=sc)
+    assert np.abs(out[0, 0, 0] - 0.5 * (v[0, 17, 0] + v[0, 23, 0])).max() < 1e-14
+    assert abs(lse[0, 0, 0] - (150.0 + math.log(2.0))) < 1e-12
+    # and the n-block merge stays exact when the blocks' maxima differ by 150 to 370
+    # natural-log units
+    O, L = oracle.block_partials(q, k, v, 4, scale=sc)
+    out_m, lse_m = oracle.merge_partials(O, L)
+    assert np.abs(out_m - out).max() < 1e-14 and np.abs(lse_m - lse).max() < 1e-12
+
+
 def test_rows_sum_to_one():
     q, k, v = _qkv(S_Q=7, S_KV=31)
     for causal in (False, True):
