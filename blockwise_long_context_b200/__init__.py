@@ -9,13 +9,16 @@ device memory and streams.  There is no fallback: if the library is missing
 every call raises.
 
 ``inputs`` (seeded synthetic workloads) imports without the library.
+``distributed`` (LV-XAttn's exchange across ranks) and ``ring`` (Ring
+Attention pass-KV) drive the same entry points over ``torch.distributed``.
 """
 
 from __future__ import annotations
 
 __all__ = [
-    "LvxError", "lib", "lvx_attn_fwd", "lvx_attn_bwd", "lvx_kv_recompute", "lvx_kv_recompute_bwd",
-    "lvx_merge_partials", "lvx_attn_fwd_noalloc", "lvx_attn_fwd_workspace", "lvx_attn_bwd_workspace",
+    "LvxError", "lib", "lvx_attn_fwd", "lvx_attn_bwd", "lvx_attn_bwd_accumulate",
+    "lvx_kv_recompute", "lvx_kv_recompute_bwd", "lvx_merge_partials", "lvx_attn_fwd_partials",
+    "lvx_attn_fwd_noalloc", "lvx_attn_fwd_workspace", "lvx_attn_bwd_workspace",
     "lvx_last_device_error", "lvx_status_string", "LVX_FP32", "LVX_BF16",
 ]
 
