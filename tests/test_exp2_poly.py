@@ -102,3 +102,47 @@ def test_packed_version_uses_the_same_clamp_and_coefficients():
     assert f"fmaxf(x0, {lo:.0f}.f)" in body and f"fmaxf(x1, {lo:.0f}.f)" in body
     nums = sorted({np.float32(v.rstrip("f")) for v in re.findall(r"-?\d\.\d+e[-+]\d+f", body)})
     assert np.array_equal(np.sort(_coefficients()), np.array(nums, dtype=np.float32))
+
+
+def _accept(x, c, lo, poly_every=4, factor=256.0, threshold=8.0):
+    """The forward kernel's steady-state acceptance of one row's 128 arguments
+    x (log2 units, relative to the running maximum): pair i of each 32-key chunk
+    goes through the FMA-pipe exponential when i % poly_every == poly_every - 1,
+    the others through the SFU (exact 2^x here; ex2.approx is within 2 ulp).
+    Accepted iff the sum of the exponentials is <= 2^threshold and every
+    FMA-pipe argument is <= threshold."""
+    x = np.asarray(x, dtype=np.float32)
+    pair = (np.arange(128) % 32) // 2
+    on_poly = pair % poly_every == poly_every - 1
+    with np.errstate(invalid="ignore", over="ignore"):     # 2^x overflows to inf, as on the SFU
+        e = np.where(on_poly, _emulate(x, c, lo), np.exp2(x.astype(np.float64)).astype(np.float32))
+        total = np.float32(e.astype(np.float32).sum(dtype=np.float32))
+        xp = np.max(np.where(on_poly, x, -np.inf))
+        return bool(total <= factor and xp <= threshold)
+
+
+def test_steady_state_acceptance_never_admits_an_exponential_above_the_threshold():
+    c, lo = _coefficients(), _clamp()
+    rng = np.random.default_rng(5)
+    pair = (np.arange(128) % 32) // 2
+    poly_keys = np.nonzero(pair % 4 == 3)[0]
+    sfu_keys = np.nonzero(pair % 4 != 3)[0]
+    rows = []
+    for _ in range(3000):                                   # ordinary rows around the maximum
+        rows.append(rng.normal(-3.0, 2.0, 128))
+    for big in (8.5, 20.0, 127.0, 128.7, 150.0, 1e4):       # one large argument on each pipe
+        for keys in (poly_keys, sfu_keys):
+            r = rng.normal(-5.0, 1.0, 128)
+            r[rng.choice(keys)] = big
+            rows.append(r)
+    rows.append(np.full(128, 7.9))                           # all just under the threshold
+    r = rng.normal(-5.0, 1.0, 128); r[3] = np.nan; rows.append(r)
+    accepted = 0
+    for r in rows:
+        if _accept(r, c, lo):
+            accepted += 1
+            assert np.nanmax(r) <= 8.0, r[np.argmax(r)]     # no exponential above 2^8
+    assert accepted >= 2900                                  # the ordinary rows pass
+    # a row the sum rejects although every argument is below the threshold falls
+    # back to the exact path (never a wrong accept, only a slower tile)
+    assert not _accept(np.full(128, 7.9), c, lo)
