@@ -10,12 +10,19 @@ S_Q=2048, S_KV=65536, n=8 KV blocks, bf16):
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lvx|reference]
 
-Prints one JSON line (rank 0).  ``value`` is whole-job TFLOP/s over all
-ranks: counted FLOPs (attention forward 4*B*H*S_Q*S_KV*d, backward 2.5x that,
-K/V recomputation 2*2*B*S_KV*d_embed*H_kv*d) divided by the max-over-ranks
-device time of K steps.  With N > 1 every rank runs its own batch of the same
+Prints one JSON line (rank 0).  ``value`` is whole-job attention TFLOP/s
+over all ranks: the attention FLOPs (forward 4*B*H*S_Q*S_KV*d, backward 2.5x
+that) divided by the device time of the attention stages (block partials +
+merge, and the backward), summed over the K timed steps and maxed over
+ranks.  The K/V recomputation (2*2*B*S_KV*d_embed*H_kv*d) runs in every step
+and is reported as its own stage; ``step_tflops`` divides all counted FLOPs
+by the whole step.  With N > 1 every rank runs its own batch of the same
 shape (weak scaling, no data-path collective).  ``--impl reference`` times
 the fp64 CPU oracle on a bounded sample of the same workload.
+
+Peaks: the measured cuBLAS bf16 burst figure for a timed region shorter than
+two seconds (the kernels then run near the maximum clock, as the burst GEMM
+did), the sustained figure (measured under the power cap) for longer ones.
 """
 
 from __future__ import annotations
@@ -50,10 +57,33 @@ TRAFFIC = {
 def _peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
-        d = json.load(open(path))
+        with open(path) as f:
+            d = json.load(f)
+        mhz = (d.get("clocks_under_load") or {}).get("sm_mhz_median")
         return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sust=d["bf16_tflops_sustained"],
-                    src="measured")
-    return dict(hbm=6650.0, bf16=1590.0, bf16_sust=1400.0, src="fallback")
+                    sust_mhz=mhz, src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sust=1400.0, sust_mhz=1300.0, src="fallback")
+
+
+# A timed region at least this long holds the power cap (as the sustained GEMM
+# measurement did); a shorter one runs near the maximum clock (as the burst did).
+SUSTAINED_AFTER_S = 2.0
+
+
+def bf16_peak(peaks, timed_s: float):
+    """(peak TFLOP/s, description) for a tensor-bound stage timed over ``timed_s`` seconds."""
+    if timed_s >= SUSTAINED_AFTER_S:
+        return peaks["bf16_sust"], (f"{peaks['src']} sustained cuBLAS bf16 (timed region "
+                                    f"{timed_s:.2f} s >= {SUSTAINED_AFTER_S} s; that peak was "
+                                    f"measured at a median {peaks['sust_mhz']} MHz)")
+    return peaks["bf16"], (f"{peaks['src']} burst cuBLAS bf16 (timed region {timed_s:.2f} s < "
+                           f"{SUSTAINED_AFTER_S} s)")
+
+
+def stats(xs):
+    """mean, median, min and max of a list of stage times (ms)."""
+    return {"mean": statistics.mean(xs), "median": statistics.median(xs), "min": min(xs),
+            "max": max(xs)}
 
 
 # ---------------------------------------------------------------- clocks
@@ -140,6 +170,8 @@ def oracle_sample(w, kv_grads: bool = False):
     if w.backward:
         oracle.attention_bwd(q, k, v, do, causal=sw.causal)
         flops += 2.5 * sw.fwd_flops()
+    t_attn = time.perf_counter() - t0
+    attn_flops = flops
     if kvw is not None:
         y = np.random.default_rng(0).standard_normal((rows, w.d_embed))
         oracle.kv_recompute(y, kvw["w_k"].double().numpy(), kvw["w_v"].double().numpy())
@@ -153,9 +185,10 @@ def oracle_sample(w, kv_grads: bool = False):
     desc = (f"fp64 oracle, forward{' + backward' if w.backward else ''} for {rows} of {w.S_Q} "
             f"query rows over all {w.H} heads and "
             f"{'all ' + str(w.S_KV) if keys == w.S_KV else f'the first {keys} of {w.S_KV}'} keys"
-            f"{f', plus K/V recompute of {rows} rows of y' if kvw is not None else ''}"
-            f"{' and its gradients' if kv_grads and kvw is not None else ''}; counted FLOPs / time")
-    return flops / dt / 1e12, dt, cores, desc
+            f"{f' (plus K/V recompute of {rows} rows of y' if kvw is not None else ''}"
+            f"{' and its gradients' if kv_grads and kvw is not None else ''}"
+            f"{', timed apart' if kvw is not None else ''}); attention FLOPs / attention time")
+    return attn_flops / t_attn / 1e12, dt, cores, desc
 
 
 def run_reference(a):
@@ -201,11 +234,11 @@ def _config(w, n, kv_grads=False):
          "l2": (f"inputs larger than L2 (126 MB): {_input_bytes(w) / 2**20:.0f} MiB read every step"
                 + (", K/V 256 MiB rewritten" if w.d_embed else "")) if _input_bytes(w) > 126e6
                else f"inputs ({_input_bytes(w) / 2**20:.1f} MiB) fit in L2: not a timing workload",
-         "flops_counted": "attn fwd 4*B*H*S_Q*S_KV*d + bwd 2.5x fwd + K/V recompute "
-                          "2*2*B*S_KV*d_embed*H_kv*d"}
+         "flops_counted": "value: attention fwd 4*B*H*S_Q*S_KV*d + bwd 2.5x fwd; step_tflops "
+                          "adds the K/V recompute 2*2*B*S_KV*d_embed*H_kv*d"}
     if kv_grads:
         c["kv_grads"] = True
-        c["flops_counted"] += " + its gradients dW_k, dW_v, dy 2x the recompute"
+        c["flops_counted"] += " and its gradients dW_k, dW_v, dy (2x the recompute)"
     return c
 
 
@@ -320,17 +353,22 @@ def run_gpu(a):
     if world > 1:
         dist.barrier()
     ms_total = e0.elapsed_time(e1)
-    t_kv = statistics.mean(ev[0].elapsed_time(ev[1]) for ev in stage_ev)
-    t_fwd = statistics.mean(ev[1].elapsed_time(ev[2]) for ev in stage_ev)
-    t_bwd = statistics.mean(ev[2].elapsed_time(ev[3]) for ev in stage_ev)
-    t_kvb = statistics.mean(ev[3].elapsed_time(ev[4]) for ev in stage_ev)
+    per = {name: [ev[i].elapsed_time(ev[i + 1]) for ev in stage_ev]
+           for i, name in enumerate(("kv", "fwd", "bwd", "kv_bwd"))}
+    t_kv, t_fwd, t_bwd, t_kvb = (statistics.mean(per[s_]) for s_ in ("kv", "fwd", "bwd", "kv_bwd"))
     lvx.lvx_last_device_error()
 
     ms_total = max_over_ranks(ms_total, dev)
     ms_step = ms_total / a.steps
     kvb_flops = 2.0 * w.kv_flops() if kv_grads else 0.0
-    step_flops = w.fwd_flops() + w.bwd_flops() + w.kv_flops() + kvb_flops
-    value = whole_job_tflops(step_flops, a.steps, world, ms_total)
+    attn_flops = w.fwd_flops() + w.bwd_flops()
+    step_flops = attn_flops + w.kv_flops() + kvb_flops
+    # attention stages only (block partials + merge, backward), summed over the
+    # timed steps, slowest rank
+    ms_attn = max_over_ranks(sum(per["fwd"]) + sum(per["bwd"]), dev)
+    value = whole_job_tflops(attn_flops, a.steps, world, ms_attn)
+    step_value = whole_job_tflops(step_flops, a.steps, world, ms_total)
+    peak_tf, peak_desc = bf16_peak(peaks, ms_total * 1e-3)
 
     # merge kernel alone (HBM-bound) through the merge entry point: ten back-to-back
     # launches per timing after an L2 flush; the partials they stream (288 MB at C1's
@@ -437,9 +475,11 @@ def run_gpu(a):
     torch.cuda.synchronize()
     ms_e2e = x0.elapsed_time(x1)
     ms_e2e = max_over_ranks(ms_e2e, dev)
-    e2e_value = whole_job_tflops(step_flops, n_e2e, world, ms_e2e)
+    # the same metric (attention FLOPs) over the whole end-to-end step: copies, K/V
+    # recomputation and attention
+    e2e_value = whole_job_tflops(attn_flops, n_e2e, world, ms_e2e)
 
-    # roofline of the dominant kernel group (timed inside the long step loop: sustained peak)
+    # roofline of the dominant kernel group, against the peak the timed region's length calls for
     stages = {"bwd": (t_bwd, w.bwd_flops(), "lvx_attn_bwd (preprocess + main + dQ finalize)"),
               "fwd": (t_fwd, w.fwd_flops(), "lvx_attn_fwd (block partials + merge)"),
               "kv": (t_kv, w.kv_flops(), "lvx_kv_recompute"),
@@ -454,25 +494,33 @@ def run_gpu(a):
     # bwd preprocess + main + dQ finalize (3)
     launches_per_step = (1 if recompute else 0) + 1 + (1 if w.n_blocks > 1 else 0) + \
         (3 if w.backward else 0) + (2 if kv_grads else 0)
+    stage_names = {"kv": "kv_recompute", "fwd": "fwd", "bwd": "bwd", "kv_bwd": "kv_recompute_bwd"}
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": a.steps,
         "warmup": warm, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded Gaussian, shapes of the "
         "pages' Llama-3-V cross-attention workload)",
         "config": _config(w, world, kv_grads),
-        "pct_of_peak": 100.0 * value / peaks["bf16_sust"],
-        "stages_ms": {"kv_recompute": t_kv, "fwd": t_fwd, "bwd": t_bwd,
-                      **({"kv_recompute_bwd": t_kvb} if kv_grads else {})},
-        "stage_tflops": {s_: (stages[s_][1] / (stages[s_][0] * 1e-3) / 1e12 if stages[s_][0] else None)
-                         for s_ in stages},
+        "pct_of_peak": 100.0 * value / peak_tf,
+        "value_counts": "attention forward (partials + merge) + backward FLOPs over their own "
+                        "stage times; the K/V recomputation is the kv_recompute stage",
+        "attn_ms_per_step": ms_attn / a.steps,
+        "step_tflops": step_value,
+        "stages_ms": {stage_names[s_]: stats(per[s_]) for s_ in stages},
+        "stage_tflops": {stage_names[s_]: (stages[s_][1] / (stages[s_][0] * 1e-3) / 1e12
+                                           if stages[s_][0] else None) for s_ in stages},
         "roofline": {"bound": "tensor", "kernel": dom_desc, "achieved": achieved,
-                     "peak": peaks["bf16_sust"], "unit": "TFLOP/s",
-                     "frac": achieved / peaks["bf16_sust"], "traffic": traffic,
-                     "peak_source": f"{peaks['src']} (sustained cuBLAS bf16, MEASURED_PEAKS.json)"},
+                     "peak": peak_tf, "unit": "TFLOP/s",
+                     "frac": achieved / peak_tf, "traffic": traffic,
+                     "achieved_from": "algorithmic FLOPs / mean CUDA-event time of the stage over "
+                                      "the timed steps",
+                     "peak_source": peak_desc + ", MEASURED_PEAKS.json"},
         "merge": {"ms": t_merge, "achieved_gbs": merge_gbs, "peak_gbs": peaks["hbm"],
                   "frac": merge_gbs / peaks["hbm"], "bytes": merge_bytes},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": n_e2e,
+                "d2h_bytes_per_step": d2h, "steps": n_e2e, "ms_per_step": ms_e2e / n_e2e,
+                "counts": "attention FLOPs over the whole step: uploads, K/V recompute, "
+                          "attention, downloads",
                 "note": ("one input set: each upload follows the previous step's compute" if single
                          else "uploads of step i+1 and downloads of step i-1 overlap step i's compute")},
         "gpu_launches": launches_per_step * a.steps,

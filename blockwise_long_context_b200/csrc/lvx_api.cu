@@ -17,10 +17,6 @@ unsigned int* device_error_word() {
   return reinterpret_cast<unsigned int*>(ptr);
 }
 
-namespace {
-
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
 lvx_status check_shapes(int B, int H, int H_kv, int S_Q, int S_KV, int d, int n_blocks,
                         int causal, lvx_dtype dt) {
   if (B < 1 || H < 1 || H_kv < 1 || S_Q < 1 || S_KV < 1 || d < 1 || n_blocks < 1)
@@ -51,6 +47,25 @@ size_t fwd_parts_o_bytes(int B, int H, int S_Q, int d, int n) {
 size_t fwd_parts_l_bytes(int B, int H, int S_Q, int n) {
   return align256((size_t)n * B * H * S_Q * sizeof(float));
 }
+
+cudaError_t run_attn_fwd(const Problem& p, lvx_dtype dt, const void* q, const void* k,
+                         const void* v, void* out, float* lse, float* o_parts, float* l_parts,
+                         cudaStream_t s) {
+  if (p.n_blocks == 1) o_parts = l_parts = nullptr;   // one block: the output directly
+  cudaError_t e;
+  if (dt == LVX_BF16 && tc_fwd_supported(p)) {
+    e = launch_fwd_tc(p, q, k, v, out, lse, o_parts, l_parts, s);
+  } else {
+    e = launch_fwd_simt(p, dt, q, k, v, out, lse, o_parts, l_parts, s);
+  }
+  if (e != cudaSuccess || p.n_blocks == 1) return e;
+  return launch_merge(o_parts, l_parts, out, lse, p.n_blocks, p.B, p.H, p.S_Q, p.d, p.causal,
+                      p.block_len, dt, s);
+}
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 lvx_status from_cuda(cudaError_t e) { return e == cudaSuccess ? LVX_OK : LVX_ERR_CUDA; }
 
@@ -97,7 +112,6 @@ lvx_status lvx_attn_fwd(const void* q, const void* k, const void* v, void* out, 
   if (!(scale == scale)) return LVX_ERR_INVALID_ARG;   // NaN scale
 
   const Problem p = make_problem(B, H, H_kv, S_Q, S_KV, d, n_blocks, causal, scale);
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   float* o_parts = nullptr;
   float* l_parts = nullptr;
   if (n_blocks > 1) {
@@ -105,17 +119,8 @@ lvx_status lvx_attn_fwd(const void* q, const void* k, const void* v, void* out, 
     l_parts = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) +
                                        fwd_parts_o_bytes(B, H, S_Q, d, n_blocks));
   }
-  cudaError_t e;
-  if (dt == LVX_BF16 && tc_fwd_supported(p)) {
-    e = launch_fwd_tc(p, q, k, v, out, lse, o_parts, l_parts, s);
-  } else {
-    e = launch_fwd_simt(p, dt, q, k, v, out, lse, o_parts, l_parts, s);
-  }
-  if (e != cudaSuccess) return LVX_ERR_CUDA;
-  if (n_blocks > 1)
-    e = launch_merge(o_parts, l_parts, out, lse, n_blocks, B, H, S_Q, d, p.causal, p.block_len,
-                     dt, s);
-  return from_cuda(e);
+  return from_cuda(run_attn_fwd(p, dt, q, k, v, out, lse, o_parts, l_parts,
+                                reinterpret_cast<cudaStream_t>(stream)));
 }
 
 lvx_status lvx_attn_fwd_partials(const void* q, const void* k, const void* v, float* O_parts,

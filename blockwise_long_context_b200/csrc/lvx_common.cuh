@@ -54,6 +54,23 @@ template <> struct Elem<__nv_bfloat16> {
 // Offsets of the two forward workspace parts (bytes).
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Argument checks, problem set-up and dispatch shared by the forward entry
+// points (defined in lvx_api.cu).
+lvx_status check_shapes(int B, int H, int H_kv, int S_Q, int S_KV, int d, int n_blocks,
+                        int causal, lvx_dtype dt);
+Problem make_problem(int B, int H, int H_kv, int S_Q, int S_KV, int d, int n_blocks, int causal,
+                     float scale);
+// Bytes of the two parts of the forward workspace: O_i [n,B,H,S_Q,d] fp32,
+// then L_i [n,B,H,S_Q] fp32, each rounded up to 256 bytes.
+size_t fwd_parts_o_bytes(int B, int H, int S_Q, int d, int n);
+size_t fwd_parts_l_bytes(int B, int H, int S_Q, int n);
+// The forward of a validated problem: block partials into o_parts / l_parts
+// and their merge (with one block, the output directly; the partials are then
+// unused and may be null).
+cudaError_t run_attn_fwd(const Problem& p, lvx_dtype dt, const void* q, const void* k,
+                         const void* v, void* out, float* lse, float* o_parts, float* l_parts,
+                         cudaStream_t s);
+
 // Launchers implemented in the kernel translation units.  Each returns the
 // cudaError_t of its launch.
 cudaError_t launch_fwd_simt(const Problem& p, lvx_dtype dt, const void* q, const void* k,

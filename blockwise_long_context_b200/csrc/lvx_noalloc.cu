@@ -20,9 +20,13 @@
 //     Nothing in it has to start at zero (every partial the merge reads is
 //     written by the same call first), but two calls whose kernels overlap
 //     on the GPU (different streams, no ordering between them) race on it.
-// The device address of the array is looked up with cudaGetSymbolAddress on
-// the first call on each device (with that device current) and cached; that
-// first call should come before any stream capture.
+// The device address of the array is looked up with cudaGetSymbolAddress the
+// first time the entry point runs in a CUDA context (the device's primary
+// context, normally) with that context current, and cached per context, so
+// a context created later (after cudaDeviceReset, say) looks it up afresh.
+// That first call should come before any stream capture.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "lvx_common.cuh"
@@ -32,32 +36,67 @@ namespace lvx {
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;
-constexpr int kMaxDevices = 64;
+constexpr int kMaxContexts = 64;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-std::mutex g_scratch_mu;
-void* g_scratch_addr[kMaxDevices] = {};
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
 
-// Device address of g_noalloc_scratch on the current device (host code must
+std::mutex g_scratch_mu;
+CtxGetCurrentFn g_ctx_current = nullptr;
+CtxGetIdFn g_ctx_id = nullptr;
+bool g_resolved = false;
+// (context id, device address of g_noalloc_scratch in that context)
+unsigned long long g_ctx_ids[kMaxContexts] = {};
+void* g_ctx_addr[kMaxContexts] = {};
+int g_n_ctx = 0;
+
+template <typename F>
+F driver_fn(const char* name) {
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &fn, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<F>(fn);
+}
+
+// Device address of g_noalloc_scratch in the current context (host code must
 // not use the symbol itself: on the host it names a stand-in, not device memory).
 cudaError_t scratch_address(void** out) {
   int dev = -1;
-  cudaError_t e = cudaGetDevice(&dev);
+  cudaError_t e = cudaGetDevice(&dev);   // also makes the device's primary context current
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_addr[dev] == nullptr) {
-    void* ptr = nullptr;
-    e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
-    if (e != cudaSuccess) return e;
-    g_scratch_addr[dev] = ptr;
+  if (!g_resolved) {
+    g_ctx_current = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+    g_ctx_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+    g_resolved = true;
   }
-  *out = g_scratch_addr[dev];
+  unsigned long long id = 0;
+  CUcontext ctx = nullptr;
+  const bool keyed = g_ctx_current && g_ctx_id && g_ctx_current(&ctx) == CUDA_SUCCESS && ctx &&
+                     g_ctx_id(ctx, &id) == CUDA_SUCCESS;
+  if (keyed) {
+    for (int i = 0; i < g_n_ctx; ++i) {
+      if (g_ctx_ids[i] == id) {
+        *out = g_ctx_addr[i];
+        return cudaSuccess;
+      }
+    }
+  }
+  void* ptr = nullptr;
+  e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+  if (e != cudaSuccess) return e;
+  if (keyed && g_n_ctx < kMaxContexts) {   // else: looked up on every call
+    g_ctx_ids[g_n_ctx] = id;
+    g_ctx_addr[g_n_ctx] = ptr;
+    ++g_n_ctx;
+  }
+  *out = ptr;
   return cudaSuccess;
 }
-
-size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -70,31 +109,21 @@ extern "C" lvx_status lvx_attn_fwd_noalloc(const void* q, const void* k, const v
                                            float* lse, int B, int H, int H_kv, int S_Q, int S_KV,
                                            int d, int n_blocks, int causal, lvx_dtype dt,
                                            float scale, lvx_stream stream) {
-  if (B < 1 || H < 1 || H_kv < 1 || S_Q < 1 || S_KV < 1 || d < 1 || n_blocks < 1)
-    return LVX_ERR_INVALID_ARG;
-  if (H % H_kv != 0 || n_blocks > S_KV) return LVX_ERR_INVALID_ARG;
-  if (dt != LVX_FP32 && dt != LVX_BF16) return LVX_ERR_UNSUPPORTED;
-  if (d > 128 || d % 8 != 0) return LVX_ERR_UNSUPPORTED;
-  if (causal && S_Q != S_KV) return LVX_ERR_UNSUPPORTED;
-  if (n_blocks > 65535 || (long long)B * H > 65535) return LVX_ERR_UNSUPPORTED;
+  // the same checks, problem and dispatch as lvx_attn_fwd; only the partials'
+  // home differs
+  lvx_status st = check_shapes(B, H, H_kv, S_Q, S_KV, d, n_blocks, causal, dt);
+  if (st != LVX_OK) return st;
   if (!q || !k || !v || !out || !lse) return LVX_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
     return LVX_ERR_INVALID_ARG;
   if (!(scale == scale)) return LVX_ERR_INVALID_ARG;
 
   // same partial layout as the lvx_attn_fwd workspace: O parts, then L parts
-  const size_t o_bytes = round256((size_t)n_blocks * B * H * S_Q * d * sizeof(float));
-  const size_t l_bytes = round256((size_t)n_blocks * B * H * S_Q * sizeof(float));
+  const size_t o_bytes = fwd_parts_o_bytes(B, H, S_Q, d, n_blocks);
+  const size_t l_bytes = fwd_parts_l_bytes(B, H, S_Q, n_blocks);
   if (n_blocks > 1 && o_bytes + l_bytes > kNoAllocScratchBytes) return LVX_ERR_WORKSPACE;
 
-  Problem p;
-  p.B = B; p.H = H; p.H_kv = H_kv; p.S_Q = S_Q; p.S_KV = S_KV; p.d = d;
-  p.n_blocks = n_blocks;
-  p.block_len = (S_KV + n_blocks - 1) / n_blocks;
-  p.causal = causal ? 1 : 0;
-  p.scale = scale > 0.f ? scale : 1.0f / sqrtf((float)d);
-  p.scale_log2 = p.scale * 1.4426950408889634f;
-
+  const Problem p = make_problem(B, H, H_kv, S_Q, S_KV, d, n_blocks, causal, scale);
   float* o_parts = nullptr;
   float* l_parts = nullptr;
   if (n_blocks > 1) {
@@ -103,13 +132,7 @@ extern "C" lvx_status lvx_attn_fwd_noalloc(const void* q, const void* k, const v
     o_parts = reinterpret_cast<float*>(base);
     l_parts = reinterpret_cast<float*>(reinterpret_cast<char*>(base) + o_bytes);
   }
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = (dt == LVX_BF16 && tc_fwd_supported(p))
-                      ? launch_fwd_tc(p, q, k, v, out, lse, o_parts, l_parts, s)
-                      : launch_fwd_simt(p, dt, q, k, v, out, lse, o_parts, l_parts, s);
-  if (e != cudaSuccess) return LVX_ERR_CUDA;
-  if (n_blocks > 1)
-    e = launch_merge(o_parts, l_parts, out, lse, n_blocks, B, H, S_Q, d, p.causal, p.block_len,
-                     dt, s);
+  const cudaError_t e = run_attn_fwd(p, dt, q, k, v, out, lse, o_parts, l_parts,
+                                     reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? LVX_OK : LVX_ERR_CUDA;
 }

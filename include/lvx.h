@@ -121,10 +121,14 @@ lvx_status lvx_attn_fwd(const void* q, const void* k, const void* v, void* out, 
  * Every GPU that loads the library holds that array until the process exits.
  * All calls on a device share it and it keeps the last call's contents;
  * nothing in it needs to start at zero, but calls whose kernels overlap on
- * the GPU race on it, so order them on one stream.  The first call on each
- * device looks up the array's device address (cudaGetSymbolAddress, with that
- * device current) and caches it; make that first call before any stream
- * capture.  No memory is allocated or freed by this call.
+ * the GPU race on it, so order them on one stream.  The first call in each
+ * CUDA context (normally a device's primary context) looks up the array's
+ * device address (cudaGetSymbolAddress, with that context current) and caches
+ * it per context, so a context created later, after cudaDeviceReset for
+ * instance, looks it up again; make the first call in a context before any
+ * stream capture.  Validation, kernels and partial layout are those of
+ * lvx_attn_fwd, so the results are identical.  No memory is allocated or
+ * freed by this call.
  */
 lvx_status lvx_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* out, float* lse,
                                 int B, int H, int H_kv, int S_Q, int S_KV, int d,
