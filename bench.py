@@ -537,6 +537,115 @@ def run_gpu(a):
         dist.destroy_process_group()
 
 
+def run_split(a):
+    """LV-XAttn's method across the ranks of the launch (``--split kv``).
+
+    Weak scaling: every rank holds one key/value shard of the workload's size
+    (the visual sequence is W * S_KV long) and S_Q / W of the query rows; K and
+    V of the shard are recomputed from the rank's shard of y each step.  The
+    forward is the ring form (query blocks travel, partials return to their
+    owner and merge there, ``distributed.xattn_forward_ring``), the backward
+    its gradient (``distributed.xattn_backward_ring``: dQ accumulators travel
+    with their blocks, dK/dV stay with the shard).  NCCL carries the
+    transfers.  ``value`` is the attention FLOPs of the whole problem
+    (4 * B * H * S_Q * W * S_KV * d forward, 2.5x that backward) over the
+    max-over-ranks device time of the attention stages."""
+    import datetime
+    import torch
+    import torch.distributed as dist
+    from blockwise_long_context_b200 import inputs
+    from blockwise_long_context_b200 import binding as lvx
+    from blockwise_long_context_b200.distributed import (shard_bounds, xattn_backward_ring,
+                                                         xattn_forward_ring)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    w = inputs.WORKLOADS[a.workload].scaled(backward=True)
+    if a.s_kv:
+        w = w.scaled(S_KV=a.s_kv)
+    qlo, qhi = shard_bounds(w.S_Q, world, rank)
+    # this rank's inputs: its query rows and its own key/value shard (seeds offset by rank)
+    wr = w.scaled(S_Q=qhi - qlo, index=w.index + 100 * rank)
+    recompute = w.d_embed > 0
+    d = inputs.make_device(wr, tensors=("q", "do") + (("y", "w_k", "w_v") if recompute
+                                                     else ("k", "v")), device=dev)
+    if recompute:
+        k = torch.empty(w.B, w.S_KV, w.H_kv, w.d, dtype=torch.bfloat16, device=dev)
+        v = torch.empty_like(k)
+    else:
+        k, v = d["k"], d["v"]
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev: ev[0].record(stream)
+        if recompute:
+            lvx.lvx_kv_recompute(d["y"], d["w_k"], d["w_v"], k, v, w.H_kv, w.d)
+        if ev: ev[1].record(stream)
+        out, lse = xattn_forward_ring(d["q"], k, v, n_local_blocks=w.n_blocks)
+        if ev: ev[2].record(stream)
+        grads = xattn_backward_ring(d["q"], k, v, out, lse, d["do"])
+        if ev: ev[3].record(stream)
+        return grads
+
+    warm = max(a.warmup, 3)
+    for _ in range(warm):
+        step()
+    torch.cuda.synchronize()
+    lvx.lvx_last_device_error()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(a.steps)]
+    clocks = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(a.steps):
+        step(evs[i])
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    lvx.lvx_last_device_error()
+    per = {n_: [ev[i].elapsed_time(ev[i + 1]) for ev in evs] for i, n_ in enumerate(("kv", "fwd", "bwd"))}
+    ms_total = max_over_ranks(e0.elapsed_time(e1), dev)
+    ms_attn = max_over_ranks(sum(per["fwd"]) + sum(per["bwd"]), dev)
+    whole = w.scaled(S_KV=world * w.S_KV)
+    attn_flops = whole.fwd_flops() + whole.bwd_flops()
+    value = attn_flops * a.steps / (ms_attn * 1e-3) / 1e12
+    peaks = _peaks()
+    peak_tf, peak_desc = bf16_peak(peaks, ms_total * 1e-3)
+    line = {
+        "metric": "LV-XAttn attention fwd+bwd TFLOP/s across the ranks (key/value sharded)",
+        "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": a.steps, "warmup": warm,
+        "ms_per_step": ms_total / a.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded Gaussian)",
+        "config": {"workload": f"{w.name} per rank: a key/value shard of {w.S_KV} keys, "
+                               f"{w.S_Q} query rows over all ranks (ring form)",
+                   "B": w.B, "H": w.H, "H_kv": w.H_kv, "d": w.d, "S_Q": w.S_Q,
+                   "S_KV_total": world * w.S_KV, "n_local_blocks": w.n_blocks,
+                   "d_embed": w.d_embed, "parallelism": f"kv{world}",
+                   "l2": "inputs larger than L2 (K/V of the shard recomputed every step)"},
+        "pct_of_peak": 100.0 * value / (world * peak_tf),
+        "peak_source": peak_desc,
+        "stages_ms": {"kv_recompute": stats(per["kv"]), "fwd": stats(per["fwd"]),
+                      "bwd": stats(per["bwd"])},
+        # per step: K/V GEMM (1), per round the partials (1) and the backward's
+        # preprocess, main kernel and dQ finalize (3), and one merge
+        "gpu_launches": a.steps * ((1 if recompute else 0) + 4 * world + 1),
+        "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def run_ring(a):
     """Ring Attention (pass-KV), the busiest rank of a ``--ring W`` ring on one GPU.
 
@@ -655,11 +764,16 @@ def main():
                     help="time the busiest rank of a Ring Attention ring of this many ranks (one GPU)")
     ap.add_argument("--ring-layout", default="contiguous", choices=["contiguous", "zigzag"],
                     help="rows per rank: one contiguous shard, or chunks r and 2W-1-r of 2W")
+    ap.add_argument("--split", default="replicas", choices=["replicas", "kv"],
+                    help="replicas: every rank runs its own batch (default); kv: LV-XAttn across "
+                         "the ranks, one key/value shard per rank (weak scaling), NCCL exchange")
     a = ap.parse_args()
     if a.impl == "reference":
         run_reference(a)
     elif a.ring:
         run_ring(a)
+    elif a.split == "kv":
+        run_split(a)
     else:
         run_gpu(a)
 

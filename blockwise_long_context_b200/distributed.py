@@ -20,6 +20,19 @@ owner moves the same bytes (one partial per round per rank) and gives the
 same result up to the order of the rescaling.  Each rank ends with the output
 of its own query rows.
 
+Backward (the pages leave it unspecified: LV-XAttn review page, referee
+report, major comment 1; this is the textbook gradient with the global
+log-sum-exp, as in the single-GPU backward).  In the ring form the key/value
+shard stays where it is, and so do the float32 accumulators of its dK, dV;
+each query block travels again, with its dO, O and log-sum-exp and a float32
+dQ accumulator.  In round s rank r adds the contributions of the block it
+holds against its own shard (``lvx_attn_bwd_accumulate``: dQ into the
+travelling accumulator, dK and dV into its own), then passes the accumulator
+on; after the last round one more hop brings every dQ home.  In the
+all-gather form every rank holds all query rows: it computes its shard's dK,
+dV locally and its contribution to every row's dQ, and one all-reduce sums
+the dQ contributions.
+
 Only the transfers are communication; every compute step runs in the
 library's CUDA kernels, and there is no CPU path.
 """
@@ -93,7 +106,7 @@ def xattn_forward_sharded(q: torch.Tensor, k_shard: torch.Tensor, v_shard: torch
     return out, lse
 
 
-def run_xattn_ring(q, k, v, partial_fn, merge_fn, exchange):
+def run_xattn_ring(q, k, v, partial_fn, merge_fn, exchange, n_local: int = 1):
     """LV-XAttn's rotation of the query blocks (LV-XAttn review page, "What
     carries the argument"; Figure 3 / Algorithm 1).  This rank keeps k, v
     [B, S_kv_r, H_kv, d]; q [B, S_r, H, d] is its query block.  In round s it
@@ -101,12 +114,15 @@ def run_xattn_ring(q, k, v, partial_fn, merge_fn, exchange):
     that block's partial against k, v with ``partial_fn`` (signature as in
     ``ring.run_ring_forward``) and sends the partial to the block's owner,
     receiving its own block's partial from rank (r + s) mod W.  ``merge_fn``
-    merges the W partials of this rank's rows."""
+    merges the W partials of this rank's rows.  With ``n_local`` > 1 each
+    round's partial is that many block partials of the key/value shard (more
+    CTAs per round when the query blocks are short), W * n_local in all."""
     world, rank = exchange.world, exchange.rank
     B, S_r, H, d = q.shape
     q_len = exchange.lengths(S_r, q.device)
-    o_parts = torch.zeros((world, B, H, S_r, d), dtype=torch.float32, device=q.device)
-    l_parts = torch.full((world, B, H, S_r), float("-inf"), dtype=torch.float32, device=q.device)
+    nl = n_local
+    o_parts = torch.zeros((world * nl, B, H, S_r, d), dtype=torch.float32, device=q.device)
+    l_parts = torch.full((world * nl, B, H, S_r), float("-inf"), dtype=torch.float32, device=q.device)
     q_cur, in_flight = q, []
     for s in range(world):
         owner = (rank - s) % world
@@ -114,13 +130,14 @@ def run_xattn_ring(q, k, v, partial_fn, merge_fn, exchange):
         if s + 1 < world:
             handle = exchange.start([q_cur], q_len[(rank - s - 1) % world])
         if s == 0:
-            partial_fn(q_cur, k, v, o_parts[0:1], l_parts[0:1], False)
+            partial_fn(q_cur, k, v, o_parts[0:nl], l_parts[0:nl], False)
         else:
             S_o = q_cur.shape[1]
-            o_p = torch.zeros((1, B, H, S_o, d), dtype=torch.float32, device=q.device)
-            l_p = torch.full((1, B, H, S_o), float("-inf"), dtype=torch.float32, device=q.device)
+            o_p = torch.zeros((nl, B, H, S_o, d), dtype=torch.float32, device=q.device)
+            l_p = torch.full((nl, B, H, S_o), float("-inf"), dtype=torch.float32, device=q.device)
             partial_fn(q_cur, k, v, o_p, l_p, False)
-            in_flight.append(exchange.exchange([o_p, l_p], owner, [o_parts[s], l_parts[s]],
+            in_flight.append(exchange.exchange([o_p, l_p], owner, [o_parts[s * nl:(s + 1) * nl],
+                                                                   l_parts[s * nl:(s + 1) * nl]],
                                                (rank + s) % world))
         if handle is not None:
             q_cur = exchange.finish(handle)[0]
@@ -129,13 +146,96 @@ def run_xattn_ring(q, k, v, partial_fn, merge_fn, exchange):
     return merge_fn(o_parts, l_parts)
 
 
-def xattn_forward_ring(q, k_shard, v_shard, group=None, scale: float = 0.0, stream=None):
+def xattn_forward_ring(q, k_shard, v_shard, group=None, scale: float = 0.0, stream=None,
+                       n_local_blocks: int = 1):
     """Cross-attention with the query rows and the key/value sequence both
     sharded across the ranks of ``group`` (rank r holds rows
     ``shard_bounds(S, W, r)`` of each) -> out [B, S_r, H, d], lse [B, H, S_r]
-    float32 for this rank's query rows.  Non-causal."""
+    float32 for this rank's query rows.  Non-causal.  ``n_local_blocks``: block
+    partials per round (see ``run_xattn_ring``)."""
     if not q.is_cuda:
         raise RuntimeError("xattn_forward_ring runs in the CUDA library; q must be on a GPU")
     from .ring import RingExchange, kernel_merge, kernel_partial
     return run_xattn_ring(q, k_shard, v_shard, kernel_partial(scale, stream),
-                          kernel_merge(q, stream), RingExchange(group))
+                          kernel_merge(q, stream), RingExchange(group), n_local_blocks)
+
+
+def _recv_like(t: torch.Tensor, n: int, seq_dim: int = 1) -> torch.Tensor:
+    shape = list(t.shape)
+    shape[seq_dim] = n
+    return torch.empty(shape, dtype=t.dtype, device=t.device)
+
+
+def run_xattn_ring_backward(q, k, v, out, lse, do, grad_fn, exchange):
+    """LV-XAttn's backward in the ring form.  This rank keeps k, v
+    [B, S_kv_r, H_kv, d] and the float32 accumulators of their gradients; its
+    query block q [B, S_r, H, d] with out, do (same shape) and lse [B, H, S_r]
+    travels as in the forward, with a float32 dq accumulator.  In round s the
+    rank holds the block of rank (r - s) mod W and ``grad_fn(q, k, v, out, lse,
+    do, diagonal, dq, dk, dv)`` (as in ``ring.run_ring_backward``) adds that
+    block's contributions; the block's other tensors move on before the
+    compute, its dq accumulator after it, and after the last round each
+    accumulator is back with its owner.  Returns float32 (dq [B, S_r, H, d],
+    dk, dv [B, S_kv_r, H_kv, d])."""
+    world, rank = exchange.world, exchange.rank
+    q_len = exchange.lengths(q.shape[1], q.device)
+    f32 = lambda t: torch.zeros(t.shape, dtype=torch.float32, device=t.device)
+    dk, dv = f32(k), f32(v)
+    cur = [q, do, out, lse.transpose(1, 2).contiguous()]   # lse travels as [B, S, H]
+    dq = f32(q)
+    for s in range(world):
+        handle = None
+        if s + 1 < world:   # the next block: rank (r - s - 1)'s, from the previous rank
+            n_in = q_len[(rank - s - 1) % world]
+            handle = exchange.exchange(cur, (rank + 1) % world, [_recv_like(t, n_in) for t in cur],
+                                       (rank - 1) % world)
+        grad_fn(cur[0], k, v, cur[2], cur[3].transpose(1, 2).contiguous(), cur[1], False, dq, dk,
+                dv)
+        if world > 1:
+            # the accumulator follows its block; after the last round it goes home
+            n_in = q_len[(rank - s - 1) % world]
+            dq = exchange.finish(exchange.exchange([dq], (rank + 1) % world,
+                                                   [_recv_like(dq, n_in)], (rank - 1) % world))[0]
+        if handle is not None:
+            cur = exchange.finish(handle)
+    return dq, dk, dv
+
+
+def xattn_backward_ring(q, k_shard, v_shard, out, lse, do, group=None, scale: float = 0.0,
+                        stream=None):
+    """Gradients of ``xattn_forward_ring``: this rank's query rows and key/value
+    shard (rows cut with ``shard_bounds``) -> dq [B, S_r, H, d], dk, dv
+    [B, S_kv_r, H_kv, d] in the input dtype, from the forward's out and lse of
+    this rank's rows.  Non-causal."""
+    if not q.is_cuda:
+        raise RuntimeError("xattn_backward_ring runs in the CUDA library; q must be on a GPU")
+    from .ring import RingExchange, kernel_block_grad
+    dq, dk, dv = run_xattn_ring_backward(q, k_shard, v_shard, out, lse, do,
+                                         kernel_block_grad(scale, stream), RingExchange(group))
+    return dq.to(q.dtype), dk.to(k_shard.dtype), dv.to(v_shard.dtype)
+
+
+def run_xattn_sharded_backward(q, k, v, out, lse, do, grad_fn, group=None):
+    """The backward of the all-gather form: every rank holds all query rows
+    and one key/value shard.  ``grad_fn`` (as above) adds the shard's
+    contributions to float32 dq, dk, dv; one all-reduce sums dq over the
+    ranks.  Returns float32 (dq [B, S_Q, H, d], dk, dv of the shard)."""
+    f32 = lambda t: torch.zeros(t.shape, dtype=torch.float32, device=t.device)
+    dq, dk, dv = f32(q), f32(k), f32(v)
+    grad_fn(q, k, v, out, lse, do, False, dq, dk, dv)
+    world, _ = _world(group)
+    if world > 1:
+        dist.all_reduce(dq, op=dist.ReduceOp.SUM, group=group)
+    return dq, dk, dv
+
+
+def xattn_backward_sharded(q, k_shard, v_shard, out, lse, do, group=None, scale: float = 0.0,
+                           stream=None):
+    """Gradients of ``xattn_forward_sharded`` -> dq [B, S_Q, H, d] (the same on
+    every rank), dk, dv of this rank's shard, in the input dtype."""
+    if not q.is_cuda:
+        raise RuntimeError("xattn_backward_sharded runs in the CUDA library; q must be on a GPU")
+    from .ring import kernel_block_grad
+    dq, dk, dv = run_xattn_sharded_backward(q, k_shard, v_shard, out, lse, do,
+                                            kernel_block_grad(scale, stream), group)
+    return dq.to(q.dtype), dk.to(k_shard.dtype), dv.to(v_shard.dtype)

@@ -274,6 +274,8 @@ def kernel_partial(scale: float = 0.0, stream=None) -> PartialFn:
     def fn(q, k_blk, v_blk, o, l, diagonal):
         if q.shape[1] == 0 or k_blk.shape[1] == 0:
             return                      # an empty block: the partial stays (0, -inf)
+        if o.shape[0] > k_blk.shape[1]:   # more slots than keys: the rest stay (0, -inf)
+            o, l = o[:k_blk.shape[1]], l[:k_blk.shape[1]]
         # one step's slice of the partials is 16-byte aligned only if its size is;
         # the library wants aligned pointers, so short shards go through a copy
         oo = o if o.data_ptr() % 16 == 0 else torch.empty_like(o)

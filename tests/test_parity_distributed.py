@@ -1,4 +1,4 @@
-"""GPU parity of the per-shard partials and of LV-XAttn's sharded forward.
+"""GPU parity of the per-shard partials and of LV-XAttn's forward and backward across ranks.
 
 ``lvx_attn_fwd_partials`` computes one key/value shard's block partials
 (O_i, L_i) without merging them; ``distributed.xattn_forward_sharded`` runs
@@ -8,7 +8,10 @@ Algorithm 1).  Runs here get one GPU, so the several ranks are emulated in
 one process -- each shard's partials computed separately and concatenated in
 rank order, which is what the all-gather produces -- and the real
 torch.distributed path runs with a one-rank NCCL group.  Every result is
-checked against the fp64 oracle's unsplit attention.
+checked against the fp64 oracle's unsplit attention, and the backward (query
+blocks with their dQ accumulators travelling, dK/dV staying with the
+stationary shard; or, in the all-gather form, dQ contributions summed over
+the ranks) against the oracle's gradient.
 """
 
 import datetime
@@ -163,3 +166,76 @@ def test_ring_form_through_torch_distributed():
     o_ref, l_ref = _oracle(host)
     compare(out, o_ref, "bf16", "ring form, torch.distributed: O")
     compare(lse, l_ref, "bf16", "ring form, torch.distributed: LSE", rel_rms=1e-4)
+
+
+def _oracle_bwd(host):
+    q, k, v, do = (host[t].double().numpy() for t in ("q", "k", "v", "do"))
+    return oracle.attention_bwd(q, k, v, do)
+
+
+def _bwd_problem(S_Q, S_KV, H=8, H_kv=2):
+    base = inputs.WORKLOADS["C2"]
+    w = base.scaled(B=1, H=H, H_kv=H_kv, d=128, S_Q=S_Q, S_KV=S_KV, n_blocks=1, causal=False,
+                    d_embed=0)
+    return w, inputs.make(w, tensors=("q", "k", "v", "do"))
+
+
+@pytest.mark.parametrize("world,S_Q,S_KV", [(2, 300, 1024), (3, 256, 1000), (4, 12, 999)])
+def test_xattn_backward_emulated_ranks(world, S_Q, S_KV):
+    """The ring form's backward with the step the distributed driver uses: for
+    every (query block o, key/value shard r) pair, in ring order, the block's
+    contributions are added to o's travelling float32 dQ accumulator and to
+    r's stationary dK, dV accumulators.  (4, 12, ...) gives shards of 3 rows."""
+    from blockwise_long_context_b200.ring import kernel_block_grad
+    w, host = _bwd_problem(S_Q, S_KV)
+    dev = {t: x.cuda() for t, x in host.items()}
+    out, lse = lvx.attention_forward(dev["q"], dev["k"], dev["v"], 1)
+    qb = [shard_bounds(S_Q, world, r) for r in range(world)]
+    kb = [shard_bounds(S_KV, world, r) for r in range(world)]
+    rows = lambda t, b: t[:, b[0]:b[1]].contiguous()
+    q, o_, do = ([rows(t, b) for b in qb] for t in (dev["q"], out, dev["do"]))
+    ls = [lse[:, :, lo:hi].contiguous() for lo, hi in qb]
+    k, v = ([rows(t, b) for b in kb] for t in (dev["k"], dev["v"]))
+    f32 = lambda t: torch.zeros(t.shape, dtype=torch.float32, device="cuda")
+    dq, dk, dv = [f32(t) for t in q], [f32(t) for t in k], [f32(t) for t in v]
+    grad = kernel_block_grad()
+    for s in range(world):
+        for r in range(world):
+            o = (r - s) % world
+            grad(q[o], k[r], v[r], o_[o], ls[o], do[o], False, dq[o], dk[r], dv[r])
+    lvx.lvx_last_device_error()
+    torch.cuda.synchronize()
+    dq_r, dk_r, dv_r = _oracle_bwd(host)
+    compare(torch.cat(dq, 1), dq_r, "bf16", f"xattn backward x{world}: dQ")
+    compare(torch.cat(dk, 1), dk_r, "bf16", f"xattn backward x{world}: dK")
+    compare(torch.cat(dv, 1), dv_r, "bf16", f"xattn backward x{world}: dV")
+
+
+@pytest.mark.parametrize("form", ["ring", "allgather"])
+def test_xattn_backward_through_torch_distributed(form):
+    """xattn_backward_ring / xattn_backward_sharded through a one-rank NCCL
+    group, after the matching forward."""
+    import torch.distributed as dist
+    from blockwise_long_context_b200.distributed import (xattn_backward_ring,
+                                                         xattn_backward_sharded, xattn_forward_ring)
+    w, host = _bwd_problem(256, 1500, H=4, H_kv=2)
+    dev = {t: x.cuda() for t, x in host.items()}
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    os.environ["MASTER_PORT"] = str(_free_port())
+    dist.init_process_group("nccl", rank=0, world_size=1, timeout=datetime.timedelta(seconds=60),
+                            device_id=torch.device("cuda", 0))
+    try:
+        if form == "ring":
+            out, lse = xattn_forward_ring(dev["q"], dev["k"], dev["v"])
+            dq, dk, dv = xattn_backward_ring(dev["q"], dev["k"], dev["v"], out, lse, dev["do"])
+        else:
+            out, lse = xattn_forward_sharded(dev["q"], dev["k"], dev["v"], n_local_blocks=2)
+            dq, dk, dv = xattn_backward_sharded(dev["q"], dev["k"], dev["v"], out, lse, dev["do"])
+        lvx.lvx_last_device_error()
+        torch.cuda.synchronize()
+    finally:
+        dist.destroy_process_group()
+    dq_r, dk_r, dv_r = _oracle_bwd(host)
+    compare(dq, dq_r, "bf16", f"{form}, torch.distributed: dQ")
+    compare(dk, dk_r, "bf16", f"{form}, torch.distributed: dK")
+    compare(dv, dv_r, "bf16", f"{form}, torch.distributed: dV")
