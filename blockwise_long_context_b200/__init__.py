@@ -19,6 +19,8 @@ __all__ = [
     "LvxError", "lib", "lvx_attn_fwd", "lvx_attn_bwd", "lvx_attn_bwd_accumulate",
     "lvx_kv_recompute", "lvx_kv_recompute_bwd", "lvx_merge_partials", "lvx_attn_fwd_partials",
     "lvx_attn_fwd_noalloc", "lvx_attn_fwd_workspace", "lvx_attn_bwd_workspace",
+    "lvx_attn_fwd_recompute", "lvx_attn_bwd_recompute", "lvx_attn_fwd_recompute_workspace",
+    "lvx_attn_bwd_recompute_workspace",
     "lvx_last_device_error", "lvx_status_string", "LVX_FP32", "LVX_BF16",
 ]
 

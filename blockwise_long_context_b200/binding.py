@@ -47,6 +47,12 @@ _SIGS = {
                                 _c_int),
     "lvx_kv_recompute": ([_vp] * 5 + [_c_int] * 5 + [_c_int, _vp], _c_int),
     "lvx_kv_recompute_bwd": ([_vp] * 8 + [_c_int] * 5 + [_c_int, _vp], _c_int),
+    "lvx_attn_fwd_recompute_workspace": ([_c_int] * 8 + [_c_int], _c_size),
+    "lvx_attn_fwd_recompute": ([_vp] * 6 + [_c_int] * 8 + [_c_int, _c_float, _vp, _c_size, _vp],
+                               _c_int),
+    "lvx_attn_bwd_recompute_workspace": ([_c_int] * 8 + [_c_int], _c_size),
+    "lvx_attn_bwd_recompute": ([_vp] * 11 + [_c_int] * 8 + [_c_int, _c_float, _vp, _c_size, _vp],
+                               _c_int),
     "lvx_last_device_error": ([_vp], _c_int),
     "lvx_selftest_wait_timeout": ([_vp], _c_int),
 }
@@ -196,6 +202,42 @@ def lvx_kv_recompute_bwd(y, w_k, w_v, dk, dv, dy, dw_k, dw_v, stream=None) -> No
                                       _stream(stream)), "lvx_kv_recompute_bwd")
 
 
+def lvx_attn_fwd_recompute_workspace(B, H, H_kv, S_Q, S_KV, d, d_embed, n_blocks, dtype: int) -> int:
+    return lib().lvx_attn_fwd_recompute_workspace(B, H, H_kv, S_Q, S_KV, d, d_embed, n_blocks, dtype)
+
+
+def lvx_attn_bwd_recompute_workspace(B, H, H_kv, S_Q, S_KV, d, d_embed, n_blocks, dtype: int) -> int:
+    return lib().lvx_attn_bwd_recompute_workspace(B, H, H_kv, S_Q, S_KV, d, d_embed, n_blocks, dtype)
+
+
+def lvx_attn_fwd_recompute(q, y, w_k, w_v, out, lse, H_kv: int, n_blocks: int, scale: float = 0.0,
+                           workspace: Optional[torch.Tensor] = None, stream=None) -> None:
+    """q [B,S_Q,H,d], y [B,S_KV,d_embed], w [d_embed,H_kv*d] -> out like q,
+    lse [B,H,S_Q] fp32, with K, V regenerated from y one key block at a time."""
+    B, S_Q, H, d = q.shape
+    S_KV, d_embed = y.shape[1], y.shape[2]
+    ws = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().lvx_attn_fwd_recompute(_ptr(q), _ptr(y), _ptr(w_k), _ptr(w_v), _ptr(out), _ptr(lse),
+                                        B, H, H_kv, S_Q, S_KV, d, d_embed, n_blocks, _dt(q),
+                                        float(scale), _ptr(workspace), ws, _stream(stream)),
+           "lvx_attn_fwd_recompute")
+
+
+def lvx_attn_bwd_recompute(q, y, w_k, w_v, out, lse, dout, dq, dy, dw_k, dw_v, H_kv: int,
+                           n_blocks: int, scale: float = 0.0,
+                           workspace: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Gradients of attention(q, y W_k, y W_v): dq like q, dy like y (bf16), dw_k,
+    dw_v [d_embed, H_kv*d] float32, with K, V regenerated one key block at a time."""
+    B, S_Q, H, d = q.shape
+    S_KV, d_embed = y.shape[1], y.shape[2]
+    ws = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().lvx_attn_bwd_recompute(_ptr(q), _ptr(y), _ptr(w_k), _ptr(w_v), _ptr(out), _ptr(lse),
+                                        _ptr(dout), _ptr(dq), _ptr(dy), _ptr(dw_k), _ptr(dw_v), B, H,
+                                        H_kv, S_Q, S_KV, d, d_embed, n_blocks, _dt(q), float(scale),
+                                        _ptr(workspace), ws, _stream(stream)),
+           "lvx_attn_bwd_recompute")
+
+
 def lvx_last_device_error(stream=None) -> None:
     _check(lib().lvx_last_device_error(_stream(stream)), "lvx_last_device_error")
 
@@ -245,6 +287,18 @@ def kv_recompute_backward(y, w_k, w_v, dk, dv):
     dy = torch.empty_like(y); dw_k = torch.empty_like(w_k); dw_v = torch.empty_like(w_v)
     lvx_kv_recompute_bwd(y, w_k, w_v, dk, dv, dy, dw_k, dw_v)
     return dy, dw_k, dw_v
+
+
+def recompute_workspaces(q, y, H_kv: int, n_blocks: int):
+    """(forward, backward) workspaces of the recomputing entry points."""
+    B, S_Q, H, d = q.shape
+    S_KV, d_embed = y.shape[1], y.shape[2]
+    f = lvx_attn_fwd_recompute_workspace(B, H, H_kv, S_Q, S_KV, d, d_embed, n_blocks, _dt(q))
+    b = lvx_attn_bwd_recompute_workspace(B, H, H_kv, S_Q, S_KV, d, d_embed, n_blocks, _dt(q))
+    if f == 0 or b == 0:
+        raise LvxError(2, "recompute_workspaces: unsupported shape or dtype")
+    return (torch.empty(f, dtype=torch.uint8, device=q.device),
+            torch.empty(b, dtype=torch.uint8, device=q.device))
 
 
 def attention_backward(q, k, v, out, lse, dout, causal: bool = False, scale: float = 0.0):

@@ -86,6 +86,8 @@ cudaError_t launch_bwd_pre(const void* out, const void* dout, const float* lse, 
 cudaError_t launch_bwd_simt(const Problem& p, lvx_dtype dt, const void* q, const void* k,
                             const void* v, const void* dout, const float* lse, const float* ND,
                             float* dq_acc, void* dk, void* dv, bool accum, cudaStream_t s);
+// The partial of an empty key block, (O, L) = (0, -inf), over `rows` rows.
+cudaError_t launch_empty_partial(float* o_part, float* l_part, size_t rows, int d, cudaStream_t s);
 // dq = scale * dq_acc in dtype dt, or with accum dq (float32) += scale * dq_acc
 cudaError_t launch_dq_finalize(const float* dq_acc, void* dq, size_t count, float scale,
                                lvx_dtype dt, bool accum, cudaStream_t s);

@@ -13,7 +13,10 @@
 // accumulator, and four warps reading it back (one 32-lane quarter each),
 // rounding to bf16 and storing.  In batched mode a launch holds two
 // independent problems (forward K and V, or dW_k and dW_v); in segment mode a
-// single problem's K loop runs over two (A, B) pairs.
+// single problem's K loop runs over two (A, B) pairs.  With float32 outputs
+// the tile is instead added to them: each row is staged in the freed pipeline
+// buffers and added with one bulk reduce-add (used when dW is summed over the
+// key blocks of a recomputing backward).
 #include "lvx_ptx.cuh"
 #include "lvx_tc.cuh"
 
@@ -28,6 +31,7 @@ constexpr uint32_t SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*ba
 
 struct GemmArgs {
   __nv_bfloat16* out[2];   // [M][N] row-major, per problem
+  float* acc[2];           // if set: float32 [M][N] the tile is added to instead
   unsigned int* err;
   int M, N;
   int kb_seg0;             // k-blocks taken from (A0, B0); the rest from (A1, B1)
@@ -148,7 +152,37 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a0, const __grid_constant
   // the MMAs before the TMEM is released.
   const bool ok = ptx::mbar_wait(acc_full, 0, args.err, kErrTimeoutEpilogue, nullptr);
   ptx::tc_fence_after();
-  if (ok && !*abort_flag) {
+  if (ok && !*abort_flag && args.acc[0] != nullptr) {
+    // float32 rows added to the output: staged with a row pitch of 1040 bytes
+    // (the 16-byte stores of a quarter-warp then fall in different banks) in
+    // the pipeline buffers, which the MMAs no longer read, then one bulk
+    // reduce-add of 1 KiB per row
+    constexpr uint32_t PITCH = BN * 4 + 16;
+    static_assert(BM * PITCH <= STAGES * STAGE_BYTES, "staging fits the pipeline buffers");
+    const int rloc = warp * 32 + lane;
+    const int row = m0 + rloc;
+    uint8_t* stg = smem + rloc * PITCH;
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      uint32_t r[32];
+      ptx::tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + c * 32, r);
+      ptx::tmem_wait_ld();
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        *reinterpret_cast<uint4*>(stg + c * 128 + q * 16) =
+            make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
+    }
+    ptx::fence_proxy_async_smem();
+    if (row < args.M) {
+      float* dst = (z ? args.acc[1] : args.acc[0]) + (size_t)row * args.N + n0;
+      asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(
+                       reinterpret_cast<uint64_t>(dst)),
+                   "r"(ptx::smem_u32(stg)), "r"((uint32_t)(BN * 4))
+                   : "memory");
+      ptx::bulk_commit();
+      ptx::bulk_wait_read();   // the staging must stay until the copy has read it
+    }
+  } else if (ok && !*abort_flag) {
     const int row = m0 + warp * 32 + lane;
     __nv_bfloat16* out = z ? args.out[1] : args.out[0];
 #pragma unroll 1
@@ -197,7 +231,7 @@ struct Operand {
 template <bool A_MN, bool B_MN>
 cudaError_t launch_gemm(const Operand* a, const Operand* b, __nv_bfloat16* out0,
                         __nv_bfloat16* out1, int M, int N, int kb_seg0, int kb_total, int batched,
-                        cudaStream_t s) {
+                        cudaStream_t s, float* acc0 = nullptr, float* acc1 = nullptr) {
   CUtensorMap ma[2], mb[2];
   for (int i = 0; i < 2; ++i) {
     const bool okA = A_MN ? map_2d(&ma[i], a[i].base, a[i].rows, a[i].cols, 64, 64)
@@ -212,6 +246,8 @@ cudaError_t launch_gemm(const Operand* a, const Operand* b, __nv_bfloat16* out0,
   GemmArgs g;
   g.out[0] = out0;
   g.out[1] = out1;
+  g.acc[0] = acc0;
+  g.acc[1] = acc1;
   g.err = device_error_word();
   g.M = M;
   g.N = N;
@@ -263,6 +299,24 @@ cudaError_t launch_kv_gemm_bwd_tc(const void* y, const void* w_k, const void* w_
   }
   // dy = dK W_k^T + dV W_v^T: M = S, N = E, K = N per segment; A = dZ stored
   // [S][N] (K-major), B = W_z stored [E][N] (K-major)
+  const Operand a[2] = {{dk, (uint64_t)S, (uint64_t)N}, {dv, (uint64_t)S, (uint64_t)N}};
+  const Operand b[2] = {{w_k, (uint64_t)E, (uint64_t)N}, {w_v, (uint64_t)E, (uint64_t)N}};
+  return launch_gemm<false, false>(a, b, reinterpret_cast<__nv_bfloat16*>(dy), nullptr, S, E,
+                                   N / BK, 2 * (N / BK), 0, s);
+}
+
+cudaError_t launch_dw_accumulate_tc(const void* y, const void* dk, const void* dv, float* dw_k,
+                                    float* dw_v, int S, int E, int N, cudaStream_t s) {
+  // dW_z += y^T dZ: as in launch_kv_gemm_bwd_tc, the tile added to float32 outputs
+  const Operand a[2] = {{y, (uint64_t)S, (uint64_t)E}, {y, (uint64_t)S, (uint64_t)E}};
+  const Operand b[2] = {{dk, (uint64_t)S, (uint64_t)N}, {dv, (uint64_t)S, (uint64_t)N}};
+  const int kb = (S + BK - 1) / BK;
+  return launch_gemm<true, true>(a, b, nullptr, nullptr, E, N, kb, kb, 1, s, dw_k, dw_v);
+}
+
+cudaError_t launch_dy_tc(const void* w_k, const void* w_v, const void* dk, const void* dv,
+                         void* dy, int S, int E, int N, cudaStream_t s) {
+  // dy = dK W_k^T + dV W_v^T (two K segments), written in bf16
   const Operand a[2] = {{dk, (uint64_t)S, (uint64_t)N}, {dv, (uint64_t)S, (uint64_t)N}};
   const Operand b[2] = {{w_k, (uint64_t)E, (uint64_t)N}, {w_v, (uint64_t)E, (uint64_t)N}};
   return launch_gemm<false, false>(a, b, reinterpret_cast<__nv_bfloat16*>(dy), nullptr, S, E,

@@ -168,6 +168,16 @@ dq_finalize_kernel(const float* __restrict__ acc, T* __restrict__ dq, size_t cou
   }
 }
 
+// The partial of an empty key block: O = 0, L = -inf (the merge's identity).
+__global__ void __launch_bounds__(256)
+empty_partial_kernel(float* __restrict__ o, float* __restrict__ l, size_t rows, int d) {
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < rows * d; i += stride)
+    o[i] = 0.f;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < rows; i += stride)
+    l[i] = -INFINITY;
+}
+
 int grid_for(size_t work, int threads) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
@@ -205,6 +215,11 @@ cudaError_t launch_bwd_pre(const void* out, const void* dout, const float* lse, 
     bwd_pre_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>((const __nv_bfloat16*)out,
                                                        (const __nv_bfloat16*)dout, lse, ND, nlse2,
                                                        dq_acc, B, H, S_Q, d);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_empty_partial(float* o_part, float* l_part, size_t rows, int d, cudaStream_t s) {
+  empty_partial_kernel<<<grid_for(rows * d, 256), 256, 0, s>>>(o_part, l_part, rows, d);
   return cudaGetLastError();
 }
 

@@ -31,4 +31,12 @@ cudaError_t launch_kv_gemm_bwd_tc(const void* y, const void* w_k, const void* w_
                                   const void* dk, const void* dv, void* dy, void* dw_k, void* dw_v,
                                   int S, int E, int N, cudaStream_t s);
 
+// Pieces of the key-block-at-a-time recomputation: dW_k += y^T dK and
+// dW_v += y^T dV added to float32 arrays (one launch), and dy = dK W_k^T +
+// dV W_v^T written in bf16.  Same shapes and support as launch_kv_gemm_bwd_tc.
+cudaError_t launch_dw_accumulate_tc(const void* y, const void* dk, const void* dv, float* dw_k,
+                                    float* dw_v, int S, int E, int N, cudaStream_t s);
+cudaError_t launch_dy_tc(const void* w_k, const void* w_v, const void* dk, const void* dv,
+                         void* dy, int S, int E, int N, cudaStream_t s);
+
 }  // namespace lvx

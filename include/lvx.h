@@ -258,6 +258,58 @@ lvx_status lvx_kv_recompute_bwd(const void* y, const void* w_k, const void* w_v,
                                 int d_embed, int H_kv, int d, lvx_dtype dt, lvx_stream stream);
 
 /*
+ * Attention with the keys and values regenerated from the visual features one
+ * key block at a time (LV-XAttn review page, "What carries the argument" and
+ * Figure 6: one shared copy of the visual features y is kept and K = y W_k,
+ * V = y W_v are recomputed wherever they are needed, the backward pass
+ * included).  Neither call ever holds the whole K, V (or dK, dV): only one
+ * block of block_len = ceil(S_KV / n_blocks) keys, in the workspace.
+ *
+ * lvx_attn_fwd_recompute: out, lse of attention(q, y W_k, y W_v), as
+ *   lvx_kv_recompute followed by lvx_attn_fwd with the same n_blocks
+ *   computes them: for each block, K_i, V_i = y_i W_k, y_i W_v, then the
+ *   block's partials; then the merge.  Workspace:
+ *   lvx_attn_fwd_recompute_workspace(...) bytes = the partials of
+ *   lvx_attn_fwd (same layout, same place) followed by two block-sized bf16
+ *   buffers.
+ * lvx_attn_bwd_recompute: the gradients of that attention with respect to q,
+ *   y and the weights, from the forward's out and lse and dout:
+ *     dq [B, S_Q, H, d] (bf16, written)
+ *     dy [B, S_KV, d_embed] (bf16, written) = dK W_k^T + dV W_v^T
+ *     dw_k, dw_v [d_embed, H_kv*d] (float32, written) = y^T dK, y^T dV
+ *   where dK, dV are attention's key/value gradients (never stored whole).
+ *   Per block: K_i, V_i regenerated; the fused backward on the block with the
+ *   global log-sum-exp (dQ added to a float32 accumulator); dy of the block's
+ *   rows written; y_i^T dK_i, y_i^T dV_i added to dw_k, dw_v.  Workspace:
+ *   lvx_attn_bwd_recompute_workspace(...) bytes = the workspace of
+ *   lvx_attn_bwd followed by four block-sized bf16 buffers.
+ * Shapes: q, out, dout [B, S_Q, H, d]; y [B, S_KV, d_embed]; w_k, w_v
+ *   [d_embed, H_kv*d] row-major; lse [B, H, S_Q] float32 (natural log).
+ *   Non-causal.  Buffers are owned by the caller; inputs and outputs must not
+ *   overlap.  Calls are stream-ordered; nothing is allocated.
+ * Constraints (else LVX_ERR_INVALID_ARG): as lvx_attn_fwd / lvx_attn_bwd,
+ *   d_embed >= 1, pointers 16-byte aligned, workspace large enough.
+ *   LVX_ERR_UNSUPPORTED unless bf16, d in {64, 128}, d_embed % 256 == 0 and
+ *   (H_kv*d) % 256 == 0 (the tensor-core GEMMs); the workspace queries then
+ *   return 0.  Block counts leaving trailing blocks empty are allowed (their
+ *   partial is the merge's identity).  LVX_ERR_CUDA if a launch fails.
+ */
+size_t lvx_attn_fwd_recompute_workspace(int B, int H, int H_kv, int S_Q, int S_KV, int d,
+                                        int d_embed, int n_blocks, lvx_dtype dt);
+lvx_status lvx_attn_fwd_recompute(const void* q, const void* y, const void* w_k, const void* w_v,
+                                  void* out, float* lse, int B, int H, int H_kv, int S_Q,
+                                  int S_KV, int d, int d_embed, int n_blocks, lvx_dtype dt,
+                                  float scale, void* workspace, size_t ws_bytes, lvx_stream stream);
+size_t lvx_attn_bwd_recompute_workspace(int B, int H, int H_kv, int S_Q, int S_KV, int d,
+                                        int d_embed, int n_blocks, lvx_dtype dt);
+lvx_status lvx_attn_bwd_recompute(const void* q, const void* y, const void* w_k, const void* w_v,
+                                  const void* out, const float* lse, const void* dout, void* dq,
+                                  void* dy, float* dw_k, float* dw_v, int B, int H, int H_kv,
+                                  int S_Q, int S_KV, int d, int d_embed, int n_blocks,
+                                  lvx_dtype dt, float scale, void* workspace, size_t ws_bytes,
+                                  lvx_stream stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device error word of the
  * current device.  Returns LVX_ERR_DEVICE_TIMEOUT if any kernel since the last
  * call gave up on a bounded wait, LVX_ERR_CUDA if the stream reported an

@@ -23,7 +23,8 @@ def to64(t: torch.Tensor) -> np.ndarray:
     return t.detach().to("cpu", torch.float64).numpy()
 
 
-def compare(gpu, ref, dtype: str, what: str, rel_rms: float | None = None) -> dict:
+def compare(gpu, ref, dtype: str, what: str, rel_rms: float | None = None,
+            mean_abs: float | None = None, max_abs: float | None = None) -> dict:
     g = to64(gpu) if isinstance(gpu, torch.Tensor) else np.asarray(gpu, dtype=np.float64)
     r = np.asarray(ref, dtype=np.float64)
     assert g.shape == r.shape, (what, g.shape, r.shape)
@@ -38,6 +39,10 @@ def compare(gpu, ref, dtype: str, what: str, rel_rms: float | None = None) -> di
     tol = dict(TOL[dtype])
     if rel_rms is not None:
         tol["rel_rms"] = rel_rms
+    if mean_abs is not None:
+        tol["mean_abs"] = mean_abs
+    if max_abs is not None:
+        tol["max_abs"] = max_abs
     for key in ("max_abs", "mean_abs", "rel_rms"):
         assert stats[key] <= tol[key], f"{what}: {key}={stats[key]:.3e} > {tol[key]:.1e} ({stats})"
     return stats

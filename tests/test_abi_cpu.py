@@ -131,3 +131,31 @@ def _parts(**kw):
 ])
 def test_fwd_partials_rejects_invalid_arguments(kw, code):
     assert _parts(**kw) == code
+
+
+def test_recompute_entry_points_validate_before_launching():
+    """The key-block-at-a-time recomputation: workspace sizes and argument
+    checks, all on the host (no GPU needed)."""
+    L = lvx.lib()
+    bf16 = lvx.LVX_BF16
+    # B, H, H_kv, S_Q, S_KV, d, d_embed, n
+    shape = (1, 32, 8, 2048, 65536, 128, 4096, 8)
+    block_kv = 8192 * 8 * 128 * 2
+    fwd = L.lvx_attn_fwd_recompute_workspace(*shape, bf16)
+    assert fwd == L.lvx_attn_fwd_workspace(1, 32, 8, 2048, 65536, 128, 8, 0, bf16) + 2 * block_kv
+    bwd = L.lvx_attn_bwd_recompute_workspace(*shape, bf16)
+    assert bwd == L.lvx_attn_bwd_workspace(1, 32, 8, 2048, 65536, 128, 0, bf16) + 4 * block_kv
+    # unsupported: fp32, d_embed not a multiple of 256, H_kv*d not a multiple of 256
+    assert L.lvx_attn_fwd_recompute_workspace(*shape, lvx.LVX_FP32) == 0
+    assert L.lvx_attn_bwd_recompute_workspace(1, 32, 8, 2048, 65536, 128, 4000, 8, bf16) == 0
+    assert L.lvx_attn_bwd_recompute_workspace(1, 4, 1, 64, 512, 128, 512, 2, bf16) == 0
+    P = 16
+    st = L.lvx_attn_fwd_recompute(P, P, P, P, P, P, *shape, bf16, 0.0, P, fwd - 1, None)
+    assert st == 3   # LVX_ERR_WORKSPACE
+    st = L.lvx_attn_fwd_recompute(None, P, P, P, P, P, *shape, bf16, 0.0, P, fwd, None)
+    assert st == 1   # LVX_ERR_INVALID_ARG
+    st = L.lvx_attn_bwd_recompute(P, P, P, P, P, P, P, P, P, P, P, *shape, lvx.LVX_FP32, 0.0, P,
+                                  bwd, None)
+    assert st == 2   # LVX_ERR_UNSUPPORTED
+    st = L.lvx_attn_bwd_recompute(P, P, P, P, P, P, P, P, P, 8, P, *shape, bf16, 0.0, P, bwd, None)
+    assert st == 1   # misaligned dw_k
