@@ -646,6 +646,95 @@ def run_split(a):
         dist.destroy_process_group()
 
 
+def run_recompute_compare(a):
+    """``--recompute-compare``: one training step of the cross-attention layer
+    with K, V regenerated from y (LV-XAttn review page, Figure 6), two ways:
+
+      materialised: K, V = y W (whole), forward, backward (dK, dV whole), then
+                    dy, dW_k, dW_v from dK, dV (lvx_kv_recompute, lvx_attn_fwd,
+                    lvx_attn_bwd, lvx_kv_recompute_bwd);
+      block-wise:   lvx_attn_fwd_recompute and lvx_attn_bwd_recompute, which
+                    regenerate one key block's K, V at a time in each pass.
+
+    Both produce out, lse, dq, dy and the weight gradients.  Prints the time per
+    step of each (CUDA events) and the device bytes each holds beyond the
+    inputs and outputs (K, V, dK, dV and workspaces)."""
+    import torch
+    from blockwise_long_context_b200 import inputs
+    from blockwise_long_context_b200 import binding as lvx
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = inputs.WORKLOADS[a.workload].scaled(backward=True)
+    if a.s_kv:
+        w = w.scaled(S_KV=a.s_kv)
+    d = inputs.make_device(w, tensors=("q", "do", "y", "w_k", "w_v"), device=dev)
+    q, do, y, wk, wv = d["q"], d["do"], d["y"], d["w_k"], d["w_v"]
+    out = torch.empty_like(q)
+    lse = torch.empty(w.B, w.H, w.S_Q, dtype=torch.float32, device=dev)
+    dq = torch.empty_like(q)
+    dy = torch.empty_like(y)
+    # materialised
+    k = torch.empty(w.B, w.S_KV, w.H_kv, w.d, dtype=torch.bfloat16, device=dev)
+    v, dk, dv = torch.empty_like(k), torch.empty_like(k), torch.empty_like(k)
+    dwk, dwv = torch.empty_like(wk), torch.empty_like(wv)
+    fws, bws = lvx.fwd_workspace(q, k, w.n_blocks), lvx.bwd_workspace(q, k)
+    mat_bytes = 4 * k.numel() * 2 + (fws.numel() if fws is not None else 0) + bws.numel()
+
+    def materialised():
+        lvx.lvx_kv_recompute(y, wk, wv, k, v, w.H_kv, w.d)
+        lvx.lvx_attn_fwd(q, k, v, out, lse, w.n_blocks, False, 0.0, fws)
+        lvx.lvx_attn_bwd(q, k, v, out, lse, do, dq, dk, dv, False, 0.0, bws)
+        lvx.lvx_kv_recompute_bwd(y, wk, wv, dk, dv, dy, dwk, dwv)
+
+    rfws, rbws = lvx.recompute_workspaces(q, y, w.H_kv, w.n_blocks)
+    dwk32 = torch.empty(wk.shape, dtype=torch.float32, device=dev)
+    dwv32 = torch.empty_like(dwk32)
+    blk_bytes = rfws.numel() + rbws.numel()
+
+    def blockwise():
+        lvx.lvx_attn_fwd_recompute(q, y, wk, wv, out, lse, w.H_kv, w.n_blocks, workspace=rfws)
+        lvx.lvx_attn_bwd_recompute(q, y, wk, wv, out, lse, do, dq, dy, dwk32, dwv32, w.H_kv,
+                                   w.n_blocks, workspace=rbws)
+
+    res = {}
+    clocks = ClockSampler(0)
+    clocks.start()
+    for name, f in (("materialised", materialised), ("blockwise", blockwise)) * 2:
+        for _ in range(max(a.warmup, 3)):
+            f()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(a.steps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            f()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        res.setdefault(name, []).extend(ts)
+    clk = clocks.stop()
+    lvx.lvx_last_device_error()
+    flops = w.fwd_flops() + w.bwd_flops() + 3 * w.kv_flops()   # K/V once, dy and dW
+    flops_blk = flops + w.kv_flops()                            # K/V regenerated in both passes
+    line = {
+        "metric": "cross-attention training step with K, V recomputed from y: materialised vs "
+                  "block-wise regeneration",
+        "unit": "ms per step", "higher_is_better": False, "n_gpus": 1, "steps": a.steps,
+        "dtype": "bf16", "data": "synthetic (seeded Gaussian)",
+        "config": {"workload": f"{w.name}: B={w.B} H={w.H} H_kv={w.H_kv} d={w.d} S_Q={w.S_Q} "
+                               f"S_KV={w.S_KV} d_embed={w.d_embed} n_blocks={w.n_blocks}"},
+        "materialised": {"ms": stats(res["materialised"]), "transient_bytes": mat_bytes,
+                         "tflops": flops / (statistics.median(res["materialised"]) * 1e-3) / 1e12,
+                         "note": "K, V, dK, dV whole (bf16) + forward and backward workspaces"},
+        "blockwise": {"ms": stats(res["blockwise"]), "transient_bytes": blk_bytes,
+                      "tflops": flops_blk / (statistics.median(res["blockwise"]) * 1e-3) / 1e12,
+                      "note": "one block's K, V, dK, dV (bf16) + partials and dQ accumulator; "
+                              "K, V are computed twice (forward and backward)"},
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_ring(a):
     """Ring Attention (pass-KV), the busiest rank of a ``--ring W`` ring on one GPU.
 
@@ -764,6 +853,8 @@ def main():
                     help="time the busiest rank of a Ring Attention ring of this many ranks (one GPU)")
     ap.add_argument("--ring-layout", default="contiguous", choices=["contiguous", "zigzag"],
                     help="rows per rank: one contiguous shard, or chunks r and 2W-1-r of 2W")
+    ap.add_argument("--recompute-compare", action="store_true",
+                    help="time a training step with K, V materialised vs regenerated block by block")
     ap.add_argument("--split", default="replicas", choices=["replicas", "kv"],
                     help="replicas: every rank runs its own batch (default); kv: LV-XAttn across "
                          "the ranks, one key/value shard per rank (weak scaling), NCCL exchange")
@@ -772,6 +863,8 @@ def main():
         run_reference(a)
     elif a.ring:
         run_ring(a)
+    elif a.recompute_compare:
+        run_recompute_compare(a)
     elif a.split == "kv":
         run_split(a)
     else:
