@@ -61,3 +61,17 @@ def test_reference_arm_is_silent_on_other_ranks():
                           "--steps", "1", "--warmup", "0"], capture_output=True, text=True,
                          env=env, cwd=ROOT, timeout=120)
     assert out.returncode == 0 and out.stdout.strip() == ""
+
+
+def test_peak_rule_and_stage_statistics():
+    """The roofline denominator: the burst cuBLAS figure for a timed region under
+    two seconds, the sustained one for longer regions; stage statistics."""
+    sys.path.insert(0, ROOT)
+    import bench
+    peaks = dict(hbm=6000.0, bf16=1600.0, bf16_sust=1400.0, sust_mhz=1350.0, src="test")
+    assert bench.bf16_peak(peaks, 0.27)[0] == 1600.0
+    assert "burst" in bench.bf16_peak(peaks, 0.27)[1]
+    assert bench.bf16_peak(peaks, 2.0)[0] == 1400.0
+    assert "sustained" in bench.bf16_peak(peaks, 5.0)[1]
+    st = bench.stats([3.0, 1.0, 2.0, 10.0])
+    assert st == {"mean": 4.0, "median": 2.5, "min": 1.0, "max": 10.0}
