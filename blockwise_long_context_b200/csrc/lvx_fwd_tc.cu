@@ -82,15 +82,15 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;     // [K_STAGES]
+  uint64_t* k0_full = bars + 1;    // K_0
+  uint64_t* kv_full = bars + 2;    // [2]: K_{j+1} and V_j landed (step j, slot j mod 2)
   uint64_t* k_empty = bars + 4;    // [K_STAGES]
-  uint64_t* v_full = bars + 7;     // [V_STAGES]
-  uint64_t* v_empty = bars + 9;    // [V_STAGES]
-  uint64_t* s_full = bars + 11;
-  uint64_t* p_full = bars + 13;
-  uint64_t* o_done = bars + 15;
-  uint64_t* mma_drain = bars + 17;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
+  uint64_t* v_empty = bars + 7;    // [V_STAGES]
+  uint64_t* s_full = bars + 9;
+  uint64_t* p_full = bars + 11;
+  uint64_t* o_done = bars + 13;
+  uint64_t* mma_drain = bars + 15;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const Problem& p = a.p;
@@ -116,14 +116,11 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     ptx::mbar_init(q_full, 1);
-    for (int s = 0; s < K_STAGES; ++s) {
-      ptx::mbar_init(&k_full[s], 1);
-      ptx::mbar_init(&k_empty[s], 1);
-    }
-    for (int s = 0; s < V_STAGES; ++s) {
-      ptx::mbar_init(&v_full[s], 1);
-      ptx::mbar_init(&v_empty[s], 1);
-    }
+    ptx::mbar_init(k0_full, 1);
+    ptx::mbar_init(&kv_full[0], 1);
+    ptx::mbar_init(&kv_full[1], 1);
+    for (int s = 0; s < K_STAGES; ++s) ptx::mbar_init(&k_empty[s], 1);
+    for (int s = 0; s < V_STAGES; ++s) ptx::mbar_init(&v_empty[s], 1);
     for (int t = 0; t < NQT; ++t) {
       ptx::mbar_init(&s_full[t], 1);
       ptx::mbar_init(&p_full[t], 128);
@@ -154,38 +151,42 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
           for (int c = 0; c < D / 64; ++c)
             ptx::tma_load_4d(smem + L::OFF_Q + t * L::TILE + c * CHUNK, &map_q, q_full, 64 * c, h,
                              m0 + BQ * t, b);
-        int issued_k = 0, issued_v = 0;
-        auto load_k = [&](int j) -> bool {
-          const int s = j % K_STAGES;
-          if (!ptx::mbar_wait(&k_empty[s], ((j / K_STAGES) & 1) ^ 1, a.err, kErrTimeoutTma, abort_flag))
-            return false;
-          ptx::mbar_arrive_expect_tx(&k_full[s], L::TILE);
-          for (int c = 0; c < D / 64; ++c)
-            ptx::tma_load_4d(smem + L::OFF_K + s * L::TILE + c * CHUNK, &map_k, &k_full[s], 64 * c,
-                             g, kb0 + BKV * j, b);
-          issued_k = j + 1;
-          return true;
-        };
-        // order K_0, then per j: K_{j+1}, V_j -- keys run ahead of values
-        bool ok = load_k(0);
+        // K_0 on a barrier of its own, then per step j one barrier for K_{j+1} and V_j:
+        // the MMA issuer waits once per step for both (a satisfied wait still keeps the
+        // issuing thread, and with it the tensor pipe, idle for ~125 cycles).  Slot j mod 2
+        // is re-armed only after PV1 of step j-2 has read V_{j-2}, by which time the issuer
+        // has long consumed that slot's previous phase.
+        ptx::mbar_arrive_expect_tx(k0_full, L::TILE);
+        for (int c = 0; c < D / 64; ++c)
+          ptx::tma_load_4d(smem + L::OFF_K + c * CHUNK, &map_k, k0_full, 64 * c, g, kb0, b);
+        int issued = 0;   // steps whose loads were issued
+        bool ok = true;
         for (int j = 0; j < T && ok; ++j) {
-          if (j + 1 < T && !load_k(j + 1)) break;
-          const int s = j % V_STAGES;
-          if (!ptx::mbar_wait(&v_empty[s], ((j / V_STAGES) & 1) ^ 1, a.err, kErrTimeoutTma, abort_flag))
+          const bool more = j + 1 < T;
+          const int ks = (j + 1) % K_STAGES, vs = j % V_STAGES;
+          if (more && !ptx::mbar_wait(&k_empty[ks], (((j + 1) / K_STAGES) & 1) ^ 1, a.err,
+                                      kErrTimeoutTma, abort_flag))
             break;
-          ptx::mbar_arrive_expect_tx(&v_full[s], L::TILE);
+          if (!ptx::mbar_wait(&v_empty[vs], ((j / V_STAGES) & 1) ^ 1, a.err, kErrTimeoutTma, abort_flag))
+            break;
+          uint64_t* bar = &kv_full[j & 1];
+          ptx::mbar_arrive_expect_tx(bar, more ? 2 * L::TILE : L::TILE);
+          if (more) {
+            for (int c = 0; c < D / 64; ++c)
+              ptx::tma_load_4d(smem + L::OFF_K + ks * L::TILE + c * CHUNK, &map_k, bar, 64 * c, g,
+                               kb0 + BKV * (j + 1), b);
+          }
           for (int c = 0; c < D / 64; ++c)
-            ptx::tma_load_4d(smem + L::OFF_V + s * L::TILE + c * CHUNK, &map_v, &v_full[s], 64 * c,
-                             g, kb0 + BKV * j, b);
-          issued_v = j + 1;
+            ptx::tma_load_4d(smem + L::OFF_V + vs * L::TILE + c * CHUNK, &map_v, bar, 64 * c, g,
+                             kb0 + BKV * j, b);
+          issued = j + 1;
         }
         if (*abort_flag) {
           // the copies already issued must land before shared memory is released
           ptx::mbar_wait(q_full, 0, a.err, kErrTimeoutTma, nullptr);
-          for (int j = issued_k > K_STAGES ? issued_k - K_STAGES : 0; j < issued_k; ++j)
-            ptx::mbar_wait(&k_full[j % K_STAGES], (j / K_STAGES) & 1, a.err, kErrTimeoutTma, nullptr);
-          for (int j = issued_v > V_STAGES ? issued_v - V_STAGES : 0; j < issued_v; ++j)
-            ptx::mbar_wait(&v_full[j % V_STAGES], (j / V_STAGES) & 1, a.err, kErrTimeoutTma, nullptr);
+          ptx::mbar_wait(k0_full, 0, a.err, kErrTimeoutTma, nullptr);
+          for (int j = issued > 2 ? issued - 2 : 0; j < issued; ++j)
+            ptx::mbar_wait(&kv_full[j & 1], (j >> 1) & 1, a.err, kErrTimeoutTma, nullptr);
         }
       }
     } else if (warp == 1) {
@@ -236,8 +237,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
           uint32_t dVprev = dV0;   // V stage of tile j-1
           bool ok = true;
           for (int j = 0; j < T && ok; ++j) {
-            ok = ptx::mbar_wait(&k_full[j % K_STAGES], (j / K_STAGES) & 1, a.err, kErrTimeoutMma,
-                                abort_flag);
+            // K_0 has a barrier of its own; K_j (j > 0) came with V_{j-1}, waited for below
+            if (j == 0) ok = ptx::mbar_wait(k0_full, 0, a.err, kErrTimeoutMma, abort_flag);
             if (!ok) break;
             ptx::tc_fence_after();
             issue_s(0);
@@ -251,8 +252,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__
             }
             issue_s(1);
             ptx::mma_commit(&k_empty[j % K_STAGES]);
-            ok = ptx::mbar_wait(&v_full[j % V_STAGES], (j / V_STAGES) & 1, a.err, kErrTimeoutMma,
-                                abort_flag);
+            ok = ptx::mbar_wait(&kv_full[j & 1], (j >> 1) & 1, a.err, kErrTimeoutMma, abort_flag);
             if (ok) ok = ptx::mbar_wait(&p_full[0], j & 1, a.err, kErrTimeoutMma, abort_flag);
             if (!ok) break;
             ptx::tc_fence_after();
